@@ -1,0 +1,332 @@
+// librma host side: argument checks, state layout, split choice, launches.
+// The C declarations and their documentation are in include/rma.h.
+#include <cmath>
+#include <cstdio>
+#include <new>
+#include <string>
+
+#include "rma_internal.cuh"
+
+namespace rma {
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& why) {
+    g_last_error = why;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(RMA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+constexpr uint64_t kAlign = 256;
+constexpr int kMaxDecodeSplits = 64;   // must match the decode kernel's kMaxSplits
+
+uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_config(const rma_config* c) {
+    if (!c) return fail(RMA_ERR_INVALID_ARG, "config is NULL");
+    if (c->batch < 1 || c->n_layers < 1 || c->n_groups < 1)
+        return fail(RMA_ERR_INVALID_ARG, "batch, n_layers and n_groups must be >= 1");
+    if (c->ring_slots < 1 || c->bank_slots < 1 || c->pend_slots < 1)
+        return fail(RMA_ERR_INVALID_ARG, "ring_slots, bank_slots and pend_slots must be >= 1");
+    if (!(std::isfinite(c->softmax_scale) && c->softmax_scale > 0.f))
+        return fail(RMA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (c->q_per_group != kQPerGroup || c->head_dim != kHeadDim)
+        return fail(RMA_ERR_UNSUPPORTED, "this build implements q_per_group == 4 and head_dim == 256");
+    if (c->ring_slots > (1 << 20)) return fail(RMA_ERR_UNSUPPORTED, "ring_slots > 2^20");
+    if (c->bank_slots + c->pend_slots > 4096) return fail(RMA_ERR_UNSUPPORTED, "bank_slots + pend_slots > 4096");
+    if (c->batch > 65535 || c->n_groups > 65535) return fail(RMA_ERR_UNSUPPORTED, "batch or n_groups > 65535");
+    if ((int64_t)c->batch * c->n_groups > (1 << 24)) return fail(RMA_ERR_UNSUPPORTED, "batch * n_groups > 2^24");
+    return RMA_OK;
+}
+
+void compute_layout(const rma_config& c, rma_layout& L) {
+    const uint64_t lbg = (uint64_t)c.n_layers * c.batch * c.n_groups;
+    const uint64_t row = (uint64_t)c.head_dim * 2;
+    uint64_t off = 0;
+    auto take = [&](uint64_t bytes) {
+        const uint64_t o = off;
+        off = round_up(off + bytes, kAlign);
+        return o;
+    };
+    L.ring_k = take(lbg * c.ring_slots * row);
+    L.ring_v = take(lbg * c.ring_slots * row);
+    L.bank_k = take(lbg * c.bank_slots * row);
+    L.bank_v = take(lbg * c.bank_slots * row);
+    L.bank_score = take(lbg * c.bank_slots * 4);
+    L.pend_k = take(lbg * c.pend_slots * row);
+    L.pend_v = take(lbg * c.pend_slots * row);
+    L.pend_score = take(lbg * c.pend_slots * 4);
+    L.counters = take(lbg * 16);
+    L.tickets = take(lbg * 4);
+    L.status = take(4);
+    L.total_bytes = off;
+}
+
+LayerView layer_view(const State& s, int layer) {
+    const rma_config& c = s.cfg;
+    const uint64_t bg = (uint64_t)c.batch * c.n_groups;
+    const uint64_t l = (uint64_t)layer;
+    LayerView v;
+    v.ring_k = reinterpret_cast<uint16_t*>(s.base + s.lay.ring_k) + l * bg * c.ring_slots * c.head_dim;
+    v.ring_v = reinterpret_cast<uint16_t*>(s.base + s.lay.ring_v) + l * bg * c.ring_slots * c.head_dim;
+    v.bank_k = reinterpret_cast<uint16_t*>(s.base + s.lay.bank_k) + l * bg * c.bank_slots * c.head_dim;
+    v.bank_v = reinterpret_cast<uint16_t*>(s.base + s.lay.bank_v) + l * bg * c.bank_slots * c.head_dim;
+    v.bank_score = reinterpret_cast<float*>(s.base + s.lay.bank_score) + l * bg * c.bank_slots;
+    v.pend_k = reinterpret_cast<uint16_t*>(s.base + s.lay.pend_k) + l * bg * c.pend_slots * c.head_dim;
+    v.pend_v = reinterpret_cast<uint16_t*>(s.base + s.lay.pend_v) + l * bg * c.pend_slots * c.head_dim;
+    v.pend_score = reinterpret_cast<float*>(s.base + s.lay.pend_score) + l * bg * c.pend_slots;
+    v.counters = reinterpret_cast<int32_t*>(s.base + s.lay.counters) + l * bg * 4;
+    v.tickets = reinterpret_cast<uint32_t*>(s.base + s.lay.tickets) + l * bg;
+    v.status = reinterpret_cast<uint32_t*>(s.base + s.lay.status);
+    v.B = c.batch;
+    v.G = c.n_groups;
+    v.R = c.ring_slots;
+    v.A = c.bank_slots;
+    v.P = c.pend_slots;
+    return v;
+}
+
+struct Splits {
+    int ring_splits, bank_splits, ring_chunk, bank_chunk;
+};
+
+// Cut `rows` into at most `want` contiguous ranges of a multiple of 4 rows.
+void cut(int rows, int want, int& n, int& chunk) {
+    want = want < 1 ? 1 : want;
+    chunk = (rows + want - 1) / want;
+    chunk = (chunk + 3) / 4 * 4;
+    if (chunk < 4) chunk = 4;
+    n = (rows + chunk - 1) / chunk;
+}
+
+Splits decode_splits(const State& s) {
+    const rma_config& c = s.cfg;
+    int want_r = s.ring_splits_override, want_b = s.bank_splits_override;
+    if (want_r <= 0 || want_b <= 0) {
+        // enough CTAs to fill every SM several times over, without cutting
+        // rows so thin that the per-split merge dominates
+        const long units = (long)c.batch * c.n_groups;
+        const long target = (long)s.sm_count * 8;
+        long per_unit = (target + units - 1) / units;
+        if (per_unit < 2) per_unit = 2;
+        if (per_unit > 32) per_unit = 32;
+        want_r = (int)(per_unit / 2);
+        want_b = (int)(per_unit - per_unit / 2);
+    }
+    Splits sp;
+    cut(c.ring_slots, want_r, sp.ring_splits, sp.ring_chunk);
+    cut(c.bank_slots, want_b, sp.bank_splits, sp.bank_chunk);
+    return sp;
+}
+
+State* as_state(rma_state* p) { return reinterpret_cast<State*>(p); }
+const State* as_state(const rma_state* p) { return reinterpret_cast<const State*>(p); }
+
+int check_layer(const State* s, int layer) {
+    if (!s) return fail(RMA_ERR_INVALID_ARG, "state is NULL");
+    if (layer < 0 || layer >= s->cfg.n_layers) return fail(RMA_ERR_INVALID_ARG, "layer index out of range");
+    return RMA_OK;
+}
+
+}  // namespace
+}  // namespace rma
+
+using namespace rma;
+
+extern "C" {
+
+size_t rma_state_bytes(const rma_config* cfg) {
+    if (check_config(cfg) != RMA_OK) return 0;
+    rma_layout L;
+    compute_layout(*cfg, L);
+    return (size_t)L.total_bytes;
+}
+
+int rma_state_alloc(const rma_config* cfg, void* dev_buf, size_t dev_bytes, void* stream, rma_state** out) {
+    int rc = check_config(cfg);
+    if (rc != RMA_OK) return rc;
+    if (!dev_buf || !out) return fail(RMA_ERR_INVALID_ARG, "dev_buf and out must be non-NULL");
+    if (!aligned(dev_buf, kAlign)) return fail(RMA_ERR_MISALIGNED, "dev_buf must be 256-byte aligned");
+    rma_layout L;
+    compute_layout(*cfg, L);
+    if (dev_bytes < L.total_bytes)
+        return fail(RMA_ERR_BUFFER_TOO_SMALL, "state buffer smaller than rma_state_bytes()");
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the device");
+    State* s = new (std::nothrow) State;
+    if (!s) return fail(RMA_ERR_INVALID_ARG, "host allocation of the handle failed");
+    s->cfg = *cfg;
+    s->lay = L;
+    s->base = static_cast<uint8_t*>(dev_buf);
+    s->ring_splits_override = 0;
+    s->bank_splits_override = 0;
+    s->sm_count = sms;
+    e = cudaMemsetAsync(s->base + L.counters, 0, L.total_bytes - L.counters, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        delete s;
+        return cuda_fail(e, "zeroing counters");
+    }
+    *out = reinterpret_cast<rma_state*>(s);
+    return RMA_OK;
+}
+
+int rma_state_layout(const rma_state* st, rma_layout* out) {
+    if (!st || !out) return fail(RMA_ERR_INVALID_ARG, "state and out must be non-NULL");
+    *out = as_state(st)->lay;
+    return RMA_OK;
+}
+
+void rma_state_free(rma_state* st) { delete as_state(st); }
+
+int rma_workspace_bytes(const rma_state* st, int n_tok, size_t* out) {
+    if (!st || !out) return fail(RMA_ERR_INVALID_ARG, "state and out must be non-NULL");
+    const State* s = as_state(st);
+    if (n_tok == 1) {
+        const Splits sp = decode_splits(*s);
+        *out = (size_t)s->cfg.batch * s->cfg.n_groups * (sp.ring_splits + sp.bank_splits) * kPartialFloats * 4;
+        return RMA_OK;
+    }
+    if (n_tok == s->cfg.pend_slots) {
+        *out = prefill_workspace_bytes(s->cfg, n_tok);
+        return RMA_OK;
+    }
+    return fail(RMA_ERR_INVALID_ARG, "n_tok must be 1 (decode) or pend_slots (prefill)");
+}
+
+int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_splits) {
+    if (!st) return fail(RMA_ERR_INVALID_ARG, "state is NULL");
+    if (ring_splits == 0 && bank_splits == 0) {
+        as_state(st)->ring_splits_override = 0;
+        as_state(st)->bank_splits_override = 0;
+        return RMA_OK;
+    }
+    if (ring_splits < 1 || bank_splits < 1 || ring_splits + bank_splits > kMaxDecodeSplits)
+        return fail(RMA_ERR_INVALID_ARG, "splits must be >= 1 each and <= 64 together (or both 0)");
+    as_state(st)->ring_splits_override = ring_splits;
+    as_state(st)->bank_splits_override = bank_splits;
+    return RMA_OK;
+}
+
+int rma_decode_step(rma_state* st, int layer, const uint16_t* q, const uint16_t* k_cur, const uint16_t* v_cur,
+                    const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score, const float* w_g,
+                    const float* b_g, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+    State* s = as_state(st);
+    int rc = check_layer(s, layer);
+    if (rc != RMA_OK) return rc;
+    if (!q || !k_cur || !v_cur || !cand_k || !cand_v || !cand_score || !w_g || !b_g || !out || !ws)
+        return fail(RMA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    const void* a16[] = {q, k_cur, v_cur, cand_k, cand_v, w_g, out, ws};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return fail(RMA_ERR_MISALIGNED, "q, k_cur, v_cur, cand_k, cand_v, w_g, out, ws need 16-byte alignment");
+    if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
+    const Splits sp = decode_splits(*s);
+    const size_t need = (size_t)s->cfg.batch * s->cfg.n_groups * (sp.ring_splits + sp.bank_splits) * kPartialFloats * 4;
+    if (ws_bytes < need) return fail(RMA_ERR_BUFFER_TOO_SMALL, "workspace smaller than rma_workspace_bytes(st, 1)");
+    if (sp.ring_splits + sp.bank_splits > kMaxDecodeSplits) return fail(RMA_ERR_UNSUPPORTED, "too many splits");
+    DecodeArgs a;
+    a.s = layer_view(*s, layer);
+    a.q = q;
+    a.k_cur = k_cur;
+    a.v_cur = v_cur;
+    a.cand_k = cand_k;
+    a.cand_v = cand_v;
+    a.cand_score = cand_score;
+    a.w_g = w_g;
+    a.b_g = b_g;
+    a.out = out;
+    a.ws = static_cast<float*>(ws);
+    a.ring_splits = sp.ring_splits;
+    a.bank_splits = sp.bank_splits;
+    a.ring_chunk = sp.ring_chunk;
+    a.bank_chunk = sp.bank_chunk;
+    a.qscale = s->cfg.softmax_scale * 1.4426950408889634f;
+    cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching rma_decode");
+    return RMA_OK;
+}
+
+int rma_admit(rma_state* st, int layer, int force, void* stream) {
+    State* s = as_state(st);
+    int rc = check_layer(s, layer);
+    if (rc != RMA_OK) return rc;
+    if (force != 0 && force != 1) return fail(RMA_ERR_INVALID_ARG, "force must be 0 or 1");
+    cudaError_t e = launch_admit(layer_view(*s, layer), force, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching rma_admit");
+    return RMA_OK;
+}
+
+int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score, const float* w_g,
+                      const float* b_g, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+    State* s = as_state(st);
+    int rc = check_layer(s, layer);
+    if (rc != RMA_OK) return rc;
+    if (!q || !k || !v || !cand_k || !cand_v || !cand_score || !w_g || !b_g || !out || !ws)
+        return fail(RMA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    const void* a16[] = {q, k, v, cand_k, cand_v, w_g, out, ws};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return fail(RMA_ERR_MISALIGNED, "q, k, v, cand_k, cand_v, w_g, out, ws need 16-byte alignment");
+    if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
+    if (n_tok != s->cfg.pend_slots || n_tok % 32 != 0 || n_tok > s->cfg.ring_slots)
+        return fail(RMA_ERR_UNSUPPORTED, "this build needs n_tok == pend_slots, a multiple of 32, <= ring_slots");
+    if (ws_bytes < prefill_workspace_bytes(s->cfg, n_tok))
+        return fail(RMA_ERR_BUFFER_TOO_SMALL, "workspace smaller than rma_workspace_bytes(st, n_tok)");
+    PrefillArgs a;
+    a.s = layer_view(*s, layer);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.cand_k = cand_k;
+    a.cand_v = cand_v;
+    a.cand_score = cand_score;
+    a.w_g = w_g;
+    a.b_g = b_g;
+    a.out = out;
+    a.ws = static_cast<float*>(ws);
+    a.n_tok = n_tok;
+    a.qscale = s->cfg.softmax_scale * 1.4426950408889634f;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_prefill(a, cs);
+    if (e == cudaErrorNotSupported) return fail(RMA_ERR_UNSUPPORTED, "rma_prefill_block is not available in this build");
+    if (e != cudaSuccess) return cuda_fail(e, "launching rma_prefill_block");
+    e = launch_admit(a.s, 1, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the forced admit");
+    return RMA_OK;
+}
+
+int rma_get_status(rma_state* st, void* stream, uint32_t* flags) {
+    if (!st || !flags) return fail(RMA_ERR_INVALID_ARG, "state and flags must be non-NULL");
+    State* s = as_state(st);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, s->base + s->lay.status, 4, cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s->base + s->lay.status, 0, 4, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+    *flags = h;
+    return RMA_OK;
+}
+
+const char* rma_strerror(int code) {
+    switch (code) {
+        case RMA_OK: return "ok";
+        case RMA_ERR_INVALID_ARG: return "invalid argument";
+        case RMA_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case RMA_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+        case RMA_ERR_CUDA: return "CUDA error";
+        case RMA_ERR_MISALIGNED: return "misaligned pointer";
+        default: return "unknown error code";
+    }
+}
+
+const char* rma_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

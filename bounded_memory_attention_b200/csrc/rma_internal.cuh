@@ -1,0 +1,85 @@
+// Internal declarations shared by the librma translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rma.h"
+
+namespace rma {
+
+constexpr int kHeadDim = 256;        // D: elements per K/V/Q row
+constexpr int kQPerGroup = 4;        // H: query heads reading one KV group
+constexpr int kRowBytes = kHeadDim * 2;
+
+// Host-side state handle: the caller's device buffer plus its layout.
+struct State {
+    rma_config cfg;
+    rma_layout lay;
+    uint8_t* base;         // device
+    int ring_splits_override;
+    int bank_splits_override;
+    int sm_count;
+};
+
+// Per-call view of one layer of the state, with device pointers already
+// offset to that layer.  All [.][.] shapes below are [batch][n_groups].
+struct LayerView {
+    uint16_t* ring_k;      // [B][G][R][D]
+    uint16_t* ring_v;
+    uint16_t* bank_k;      // [B][G][A][D]
+    uint16_t* bank_v;
+    float* bank_score;     // [B][G][A]
+    uint16_t* pend_k;      // [B][G][P][D]
+    uint16_t* pend_v;
+    float* pend_score;     // [B][G][P]
+    int32_t* counters;     // [B][G][4] = pos, bank_fill, pend_fill, 0
+    uint32_t* tickets;     // [B][G]
+    uint32_t* status;
+    int B, G, R, A, P;
+};
+
+struct DecodeArgs {
+    LayerView s;
+    const uint16_t* q;          // [B][G*H][D]
+    const uint16_t* k_cur;      // [B][G][D]
+    const uint16_t* v_cur;
+    const uint16_t* cand_k;
+    const uint16_t* cand_v;
+    const float* cand_score;    // [B][G]
+    const float* w_g;           // [G*H][D]
+    const float* b_g;           // [G*H]
+    uint16_t* out;              // [B][G*H][D]
+    float* ws;                  // partials [B][G][splits][kPartialFloats]
+    int ring_splits, bank_splits;
+    int ring_chunk, bank_chunk; // rows per split (multiples of 4)
+    float qscale;               // softmax_scale * log2(e)
+};
+
+struct PrefillArgs {
+    LayerView s;
+    const uint16_t* q;          // [B][n][G*H][D]
+    const uint16_t* k;          // [B][n][G][D]
+    const uint16_t* v;
+    const uint16_t* cand_k;
+    const uint16_t* cand_v;
+    const float* cand_score;    // [B][n][G]
+    const float* w_g;
+    const float* b_g;
+    uint16_t* out;              // [B][n][G*H][D]
+    float* ws;
+    int n_tok;
+    float qscale;
+};
+
+// One split's partial softmax result for the 4 heads of a group:
+// m[4] (running max, log2 domain), l[4] (sum of exponentials), acc[4][D].
+constexpr int kPartialFloats = 4 + 4 + kQPerGroup * kHeadDim;
+
+// Launchers (each returns cudaGetLastError() of its launch).
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok);
+
+}  // namespace rma

@@ -1,0 +1,219 @@
+/*
+ * librma: the Rock Memory Anchors (RMA) attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * A C ABI over plain pointers and sizes.  Every device buffer is owned by the
+ * caller; the library allocates no device memory, ever.  Calls are
+ * asynchronous on the stream passed in (a cudaStream_t given as `void*`;
+ * NULL is the legacy default stream) and return before the GPU work ends.
+ *
+ * Pages the operations come from (cited by title and section):
+ *   [NEWS] "EdgeRock-4B holds KV cache at 72 MiB up to 256K context, with
+ *          12,124 tokens/s on one 80GB GPU" (tpsreport.news)
+ *   [PRIM] "EdgeRock-4B fixes its attention KV cache at 72 MiB" (ai-primer.com)
+ *   [CARD] "EdgeRock" model card (modelscope.cn/models/rockmatrix/EdgeRock)
+ *   [SITE] "Models / EdgeRock-4B" product page (rockmatrix.ai/models)
+ *
+ * State, per (sequence, RMA layer, KV group) ([CARD] "How Rock Memory Anchors
+ * work", history-component table; [PRIM] persistent-history table):
+ *   ring     R slots of (K, V)      the preceding positions of the local window
+ *                                   (position p lives in slot p mod R); the
+ *                                   decoder supplies the current token.
+ *   bank     A records (K, V, score) committed anchors, valid prefix [0, bank_fill)
+ *   pending  P records (K, V, score) candidates of the next admit, [0, pend_fill)
+ *   counters pos, bank_fill, pend_fill
+ * The pages fix R = 1023, A = 1024, P = 256, 4 KV groups, BF16 K/V; head_dim
+ * 256 and 4 query heads per group follow from the source model's 32 KiB of KV
+ * per token over 8 layers ([NEWS] "Throughput and memory").
+ *
+ * Numbers: K, V, Q and outputs are BF16, passed as their uint16_t bit
+ * patterns; scores and gate parameters are FP32; all accumulation is FP32.
+ *
+ * Error behaviour: every call returns RMA_OK (0) or a negative RMA_ERR_* code.
+ * Argument, shape, size and alignment errors are found on the host before
+ * anything is launched; rma_last_error() then gives a one-line reason.
+ * Conditions only the GPU can see never trap: they set bits in a device
+ * status word (RMA_STATUS_*), read and cleared by rma_get_status().
+ */
+#ifndef RMA_H
+#define RMA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RMA_API __attribute__((visibility("default")))
+#else
+#define RMA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ---- */
+#define RMA_OK                    0
+#define RMA_ERR_INVALID_ARG      -1  /* null pointer, bad layer index, bad flag value */
+#define RMA_ERR_UNSUPPORTED      -2  /* a shape this build does not implement */
+#define RMA_ERR_BUFFER_TOO_SMALL -3  /* state buffer or workspace smaller than required */
+#define RMA_ERR_CUDA             -4  /* a CUDA runtime call or kernel launch failed */
+#define RMA_ERR_MISALIGNED       -5  /* a pointer lacks the alignment stated below */
+
+/* ---- device status bits (rma_get_status) ---- */
+/* A decode step found the pending buffer full (rma_admit was skipped): its
+ * candidate was dropped; attention, ring write and pos advance still happened. */
+#define RMA_STATUS_PENDING_OVERFLOW          1u
+/* An admit met a NaN score; NaN ranks below every number (see rma_admit). */
+#define RMA_STATUS_NAN_SCORE                 2u
+/* A prefill block's candidates did not fit the pending buffer: they were
+ * dropped; the rest of the block (attention, ring, forced admit) ran. */
+#define RMA_STATUS_PREFILL_PENDING_OVERFLOW  4u
+/* A kernel found counters outside their ranges (pos < 0, bank_fill not in
+ * [0, bank_slots], pend_fill not in [0, pend_slots]), e.g. a corrupted restore:
+ * it clamped them for its own indexing and went on. */
+#define RMA_STATUS_BAD_COUNTERS              8u
+
+/* Dimensions.  This build implements q_per_group == 4 and head_dim == 256
+ * (RMA_ERR_UNSUPPORTED otherwise), any n_groups >= 1, ring_slots in
+ * [1, 1<<20], bank_slots >= 1, pend_slots >= 1, bank_slots + pend_slots <= 4096. */
+typedef struct rma_config {
+    int32_t batch;          /* independent sequences */
+    int32_t n_layers;       /* RMA layers (8 in the pages' model) */
+    int32_t n_groups;       /* KV groups (4) */
+    int32_t q_per_group;    /* query heads per KV group (4) */
+    int32_t head_dim;       /* D (256) */
+    int32_t ring_slots;     /* R (1023) */
+    int32_t bank_slots;     /* A (1024) */
+    int32_t pend_slots;     /* P (256) */
+    float   softmax_scale;  /* 1/sqrt(head_dim) = 1/16 */
+} rma_config;
+
+/* Byte offsets, from the start of the caller's state buffer, of each array.
+ * Every offset is a multiple of 256.  Shapes (row-major, innermost last):
+ *   ring_k, ring_v        bf16  [n_layers][batch][n_groups][ring_slots][head_dim]
+ *   bank_k, bank_v        bf16  [n_layers][batch][n_groups][bank_slots][head_dim]
+ *   bank_score            f32   [n_layers][batch][n_groups][bank_slots]
+ *   pend_k, pend_v        bf16  [n_layers][batch][n_groups][pend_slots][head_dim]
+ *   pend_score            f32   [n_layers][batch][n_groups][pend_slots]
+ *   counters              i32   [n_layers][batch][n_groups][4] = {pos, bank_fill, pend_fill, 0}
+ *   tickets               u32   [n_layers][batch][n_groups]  (library-internal, zero between calls)
+ *   status                u32   one word (RMA_STATUS_* bits)
+ * A caller may write the slot arrays and counters directly (to restore a
+ * checkpoint or set up a test) while no call is in flight. */
+typedef struct rma_layout {
+    uint64_t total_bytes;
+    uint64_t ring_k, ring_v, bank_k, bank_v, bank_score;
+    uint64_t pend_k, pend_v, pend_score, counters, tickets, status;
+} rma_layout;
+
+typedef struct rma_state rma_state;   /* opaque host handle; the device memory is the caller's */
+
+/* Bytes of device memory the state needs for cfg, or 0 if cfg is invalid.
+ * Independent of sequence length: the state has fixed capacity ([CARD]
+ * "How Rock Memory Anchors work": O(1) persistent history). */
+RMA_API size_t rma_state_bytes(const rma_config* cfg);
+
+/* Lay the state out over dev_buf (device memory, 256-byte aligned, at least
+ * rma_state_bytes(cfg) bytes, owned by the caller and kept alive until
+ * rma_state_free) and zero its counters, tickets and status word on
+ * `stream`.  Slot contents are left as they are.  Allocates no device memory.
+ * On success *out receives a host handle. */
+RMA_API int rma_state_alloc(const rma_config* cfg, void* dev_buf, size_t dev_bytes, void* stream, rma_state** out);
+
+/* Copy the layout of st into *out. */
+RMA_API int rma_state_layout(const rma_state* st, rma_layout* out);
+
+/* Release the host handle (not the caller's device buffer).  NULL is a no-op. */
+RMA_API void rma_state_free(rma_state* st);
+
+/* Workspace (device scratch, 256-byte aligned) a call with n_tok tokens per
+ * sequence needs: n_tok == 1 for rma_decode_step, n_tok == pend_slots for
+ * rma_prefill_block.  The caller owns it; its contents need not be preserved
+ * between calls, but two calls in flight at once need two workspaces. */
+RMA_API int rma_workspace_bytes(const rma_state* st, int n_tok, size_t* out);
+
+/* Decode split-K shape: the ring and the bank are each cut into this many
+ * contiguous row ranges, one CTA per range.  0 for both restores the default
+ * (chosen from batch size and SM count).  Affects speed only, not results
+ * beyond FP32 summation order. */
+RMA_API int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_splits);
+
+/* One decode token for every sequence at RMA layer `layer`
+ * ([PRIM] operations list, items 1-3; [CARD] "How Rock Memory Anchors work"):
+ *   local_h  = softmax(scale q_h K^T) V over the window: ring slots holding
+ *              positions [pos - min(pos, R), pos) plus the current token;
+ *   anchor_h = the same over bank slots [0, bank_fill) (0 if bank_fill == 0);
+ *   g_h      = tanh(q_h . w_g[h] + b_g[h]);   out_h = local_h + g_h anchor_h,
+ * for every query head h, which reads KV group h / q_per_group.  Then, after
+ * every read of the step: (k_cur, v_cur) go to ring slot pos mod R, pos += 1,
+ * and (cand_k, cand_v, cand_score) are appended at pending slot pend_fill
+ * (or dropped with RMA_STATUS_PENDING_OVERFLOW if pend_fill == P).
+ * Pending records are never read.
+ *   q          bf16 [batch][n_groups*q_per_group][head_dim]
+ *   k_cur, v_cur, cand_k, cand_v   bf16 [batch][n_groups][head_dim]
+ *   cand_score f32  [batch][n_groups]
+ *   w_g        f32  [n_groups*q_per_group][head_dim]   (this layer's)
+ *   b_g        f32  [n_groups*q_per_group]
+ *   out        bf16 [batch][n_groups*q_per_group][head_dim]   (written)
+ *   ws         workspace of rma_workspace_bytes(st, 1) bytes
+ * All pointers are device pointers; q, k_cur, v_cur, cand_k, cand_v, w_g and
+ * out must be 16-byte aligned.  Does not run the admit: call rma_admit next. */
+RMA_API int rma_decode_step(rma_state* st, int layer,
+                    const uint16_t* q, const uint16_t* k_cur, const uint16_t* v_cur,
+                    const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
+                    const float* w_g, const float* b_g, uint16_t* out,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Admit at RMA layer `layer` ([NEWS] "How it works": after every 256
+ * candidates the existing anchors and the candidates compete and the top
+ * 1,024 are kept, independently per KV group; [SITE] "Commit interval 256").
+ * For each (sequence, group) with pend_fill == P (or, when force != 0, with
+ * pend_fill > 0): the bank_fill committed records and pend_fill candidates
+ * are ordered by score (higher first), then committed before candidate, then
+ * lower slot (-0.0 equals +0.0; NaN below every number, and it sets
+ * RMA_STATUS_NAN_SCORE); the first min(A, bank_fill + pend_fill) are kept.
+ * Retained anchors stay in their slots, unchanged ([PRIM] item 3).  Admitted
+ * candidates, in ascending pending slot, are copied (K, V and score,
+ * bit-exact) into the vacated slots (evicted anchors' slots and empty slots)
+ * in ascending order.  Then bank_fill = number kept, pend_fill = 0.
+ * Other (sequence, group) pairs are untouched.  force must be 0 or 1. */
+RMA_API int rma_admit(rma_state* st, int layer, int force, void* stream);
+
+/* A prefill block of n_tok consecutive tokens per sequence at RMA layer
+ * `layer` ([CARD] FAQ "How do Rock Memory Anchors preserve distant
+ * information?": reads use the committed bank; updates take effect at the
+ * next block).  With block start s = pos, query i (position s + i) attends
+ * causally to positions [s + i - R, s + i] (ring slots for those below s, the
+ * block's own k, v for the rest) and to bank slots [0, bank_fill) as
+ * committed before the block; gate and output as in rma_decode_step.  Then,
+ * after every read: ring slots (s + i) mod R take k, v of the block, pos +=
+ * n_tok, the candidates are appended to pending (if pend_fill + n_tok <= P,
+ * else dropped with RMA_STATUS_PREFILL_PENDING_OVERFLOW), and the admit runs
+ * forced (as rma_admit with force = 1).
+ *   q           bf16 [batch][n_tok][n_groups*q_per_group][head_dim]
+ *   k, v, cand_k, cand_v   bf16 [batch][n_tok][n_groups][head_dim]
+ *   cand_score  f32  [batch][n_tok][n_groups]
+ *   w_g, b_g    as in rma_decode_step
+ *   out         bf16 [batch][n_tok][n_groups*q_per_group][head_dim]  (written)
+ *   ws          workspace of rma_workspace_bytes(st, n_tok) bytes
+ * This build requires n_tok == pend_slots, n_tok a multiple of 32 and
+ * n_tok <= ring_slots (RMA_ERR_UNSUPPORTED otherwise).  Alignment as in
+ * rma_decode_step. */
+RMA_API int rma_prefill_block(rma_state* st, int layer, int n_tok,
+                      const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
+                      const float* w_g, const float* b_g, uint16_t* out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Wait for `stream`, then read the device status word into *flags and clear it. */
+RMA_API int rma_get_status(rma_state* st, void* stream, uint32_t* flags);
+
+/* Text for a return code. */
+RMA_API const char* rma_strerror(int code);
+
+/* One line describing the most recent error returned on this host thread ("" if none). */
+RMA_API const char* rma_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RMA_H */

@@ -123,3 +123,40 @@ def state_contents(n_layers: int, batch: int, n_groups: int, head_dim: int, ring
         "pend_v": bf16_normal((L, B, G, P, D), s + 6, device),
         "pend_score": sc((L, B, G, P), s + 7, device),
     }
+
+
+def workload_counters(kind: str, n_layers: int, batch: int, n_groups: int, ring_slots: int = 1023,
+                      bank_slots: int = 1024, pend_slots: int = 256, seed: int = 0) -> dict:
+    """Starting counters (pos, bank_fill, pend_fill), each int64 [L, B, G], for the named workloads.
+
+    tiny     ring pre-filled (pos = R), bank full, pending empty
+    batch    rings full (pos = 131072 + b mod P), banks full, pending staggered
+             at b mod P so that pos mod P == pend_fill
+    long     pos = 131072, ring and bank full, pending empty
+    ragged   per (layer, sequence): ring fill U{1..R} (pos = fill), bank fill
+             U{0..A}, pending fill U{0..P-1}
+    empty    everything zero (block prefill starts here)
+    """
+    import numpy as np
+    L, B, G, R, A, P = n_layers, batch, n_groups, ring_slots, bank_slots, pend_slots
+    shape = (L, B, G)
+    if kind == "tiny":
+        pos, bank, pend = np.full(shape, R), np.full(shape, A), np.zeros(shape)
+    elif kind == "batch":
+        b = np.arange(B)[None, :, None] % P
+        pos = np.broadcast_to(131072 + b, shape)
+        bank = np.full(shape, A)
+        pend = np.broadcast_to(b, shape)
+    elif kind == "long":
+        pos, bank, pend = np.full(shape, 131072), np.full(shape, A), np.zeros(shape)
+    elif kind == "ragged":
+        pos = uniform_int((L, B, 1), 1, R, seed * 3 + 1).numpy()
+        bank = uniform_int((L, B, 1), 0, A, seed * 3 + 2).numpy()
+        pend = uniform_int((L, B, 1), 0, P - 1, seed * 3 + 3).numpy()
+        pos, bank, pend = (np.broadcast_to(x, shape) for x in (pos, bank, pend))
+    elif kind == "empty":
+        pos = bank = pend = np.zeros(shape)
+    else:
+        raise ValueError(kind)
+    return {"pos": np.array(pos, dtype=np.int64), "bank_fill": np.array(bank, dtype=np.int64),
+            "pend_fill": np.array(pend, dtype=np.int64)}
