@@ -1,0 +1,446 @@
+"""Benchmark: RMA-layer decode tokens/s at batch 512 x 8 layers, and the HBM roofline fraction.
+
+Workload (default): 512 independent sequences, 8 RMA layers, 4 KV groups x 4
+query heads, head_dim 256, BF16 K/V; every ring full (1,023 positions) and
+every bank full (1,024 records); pending buffers staggered at fill b mod 256
+so two sequences per layer admit on every step.  One step = for each of the 8
+layers, rma_decode_step then rma_admit.  Per-step inputs (Q, current K/V,
+candidate K/V/score) come from a pool of 16 pre-generated step sets, cycled,
+so input generation is outside the timed region.  The 36 GB state is far
+larger than L2, so no flush is needed between steps.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...     (one replica per GPU)
+  python bench.py --workload long|ragged|prefill         (other workloads)
+
+Multi-GPU: sequences are independent, so each rank runs its own 512-sequence
+replica with no data-path collective ("weak" scaling); the only collectives
+are the harness's barrier and the max-over-ranks of the timed duration.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RMA-layer decode tokens/s at batch 512 x 8 layers; % of B200 HBM roofline"
+UNIT = "tokens/s"
+# algorithmic bytes per (sequence, layer, decode step) with ring and bank full:
+# ring K+V 4*1023*1024, bank K+V 4*1024*1024, q 8192, out 8192, k_cur+v_cur 4096, ring write 4096
+BYTES_FULL = 4 * 1023 * 1024 + 4 * 1024 * 1024 + 8192 + 8192 + 4096 + 4096
+FALLBACK_HBM_GBS = 6650.0
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "rma_decode_batch512.md")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "bounded_memory_attention_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(profile_path: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source.
+
+    The summary holds a line 'traffic_bytes_per_launch_batch512: <int>' and a
+    line 'kernel_source_sha256_16: <hash>'; a different hash means the kernel
+    changed since the counters were taken, and traffic is reported as null.
+    """
+    if not os.path.exists(profile_path):
+        return None
+    vals = {}
+    with open(profile_path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip().strip("`-* ")] = v.strip().strip("`* ")
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash(source):
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch_batch512"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.uuid = uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                pw.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "power_w_max": max(pw),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# workload set-up (device side)
+# ---------------------------------------------------------------------------
+
+def make_decode_workload(rma, torch, si, B: int, L: int, kind: str, seed: int, device):
+    cfg = rma.Config(batch=B, n_layers=L)
+    st = rma.State(cfg, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    for name in ("ring_k", "ring_v", "bank_k", "bank_v", "pend_k", "pend_v"):
+        getattr(st, name).normal_(generator=g)
+    if kind == "ragged":
+        for name in ("bank_score", "pend_score"):
+            z = torch.randn(getattr(st, name).shape, generator=g, device=device)
+            getattr(st, name).copy_((torch.clamp(torch.floor(4 * z) + 8, 0, 15) - 8) / 4)
+    else:
+        st.bank_score.normal_(generator=g)
+        st.pend_score.normal_(generator=g)
+    c = si.workload_counters(kind, L, B, cfg.n_groups, seed=seed)
+    cnt = torch.zeros(L, B, cfg.n_groups, 4, dtype=torch.int32)
+    cnt[..., 0] = torch.from_numpy(c["pos"])
+    cnt[..., 1] = torch.from_numpy(c["bank_fill"])
+    cnt[..., 2] = torch.from_numpy(c["pend_fill"])
+    st.counters.copy_(cnt)
+    w, b = si.gate_params(L, cfg.n_q_heads, cfg.head_dim, seed, device=device)
+    pool = [[si.decode_inputs(B, cfg.n_groups, cfg.q_per_group, cfg.head_dim, seed=1000 * s + l, device=device,
+                              quantized_scores=(kind == "ragged"))
+             for l in range(L)] for s in range(16)]
+    torch.cuda.synchronize(device)
+    return cfg, st, w, b, pool
+
+
+def step_input_bytes(B: int, L: int) -> tuple:
+    h2d = L * (B * 16 * 256 * 2 + 4 * B * 4 * 256 * 2 + B * 4 * 4)
+    d2h = L * B * 16 * 256 * 2
+    return h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle baseline
+# ---------------------------------------------------------------------------
+
+def _np(t):
+    """Torch tensor -> numpy in storage form (bf16 as uint16 bits)."""
+    import numpy as np
+    import torch
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+
+def cpu_oracle_decode(n_seq: int, n_layers: int, n_steps: int, seed: int = 0) -> dict:
+    """Time the oracle on the batch-512 workload restricted to n_seq sequences (one host thread)."""
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(batch=n_seq, n_layers=n_layers)
+    cont = si.state_contents(n_layers, n_seq, 4, 256, 1023, 1024, 256, seed=seed)
+    c = si.workload_counters("batch", n_layers, n_seq, 4)
+    st = oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, **c)
+    w, b = si.gate_params(n_layers, 16, 256, seed)
+    w, b = w.numpy(), b.numpy()
+    ins = [[{k: _np(v) for k, v in si.decode_inputs(n_seq, 4, 4, 256, seed=1000 * s + l).items()}
+            for l in range(n_layers)] for s in range(n_steps)]
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for s in range(n_steps):
+            for l in range(n_layers):
+                x = ins[s][l]
+                oracle.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"],
+                                   x["cand_score"], w[l], b[l])
+                oracle.admit(st, l)
+        dt = time.perf_counter() - t0
+    return {"value": n_seq * n_steps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n_seq} of the 512 sequences x {n_layers} layers x {n_steps} steps "
+                      f"(decode + admit), FP64 numpy oracle, 1 thread; {dt:.1f} s"}
+
+
+def run_reference(args) -> None:
+    """The reference arm: the CPU oracle as it stands, on this machine's host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # each step is a bounded sample of the batch-512 workload: one sequence x 8 layers
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    n_layers = 8
+    cfg = oracle.Config(batch=1, n_layers=n_layers)
+    n_src = 4   # sequences of the workload visited in turn
+    states = []
+    for sidx in range(n_src):
+        cont = si.state_contents(n_layers, 1, 4, 256, 1023, 1024, 256, seed=sidx)
+        c = si.workload_counters("batch", n_layers, 1, 4)
+        c["pos"] += 64 * sidx
+        c["pend_fill"] += 64 * sidx
+        states.append(oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, **c))
+    w, b = si.gate_params(n_layers, 16, 256, 0)
+    w, b = w.numpy(), b.numpy()
+    pool = [[{k: _np(v) for k, v in si.decode_inputs(1, 4, 4, 256, seed=1000 * s + l).items()}
+             for l in range(n_layers)] for s in range(16)]
+
+    def step(i):
+        st = states[i % n_src]
+        for l in range(n_layers):
+            x = pool[i % 16][l]
+            oracle.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"],
+                               x["cand_score"], w[l], b[l])
+            oracle.admit(st, l)
+
+    with threadpool_limits(limits=1):
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        dt = time.perf_counter() - t0
+    value = args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "batch-512 decode, sampled: each step is one of the 512 sequences through "
+                               "8 RMA layers (decode + admit), 4 KV groups x 4 q-heads, head_dim 256, "
+                               "full ring and bank, staggered pending"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "1 sequence x 8 layers per step (numpy FP64 oracle, 1 thread)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1024)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="batch", choices=["batch", "long", "ragged"])
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    from bounded_memory_attention_b200 import build
+    build.build()
+    import bounded_memory_attention_b200 as rma
+    import synth_inputs as si
+
+    B = args.batch or {"batch": 512, "long": 1, "ragged": 512}[args.workload]
+    L = 8
+    kind = args.workload
+    cfg, st, w, b, pool = make_decode_workload(rma, torch, si, B, L, kind, seed=rank, device=device)
+    ws = st.workspace(1)
+    out = torch.empty(B, 16, 256, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i, ev=None):
+        for l in range(L):
+            x = pool[i % 16][l]
+            if ev is not None:
+                ev[l][0].record(stream)
+            rma.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"], x["cand_score"],
+                            w[l], b[l], out, ws, stream=stream)
+            if ev is not None:
+                ev[l][1].record(stream)
+            rma.admit(st, l, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+           for _ in range(K)]
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    t0e.record(stream)
+    for i in range(K):
+        step(args.warmup + i, evs[i])
+    t1e.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t0e.elapsed_time(t1e)
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / K
+    value = world * B * K / (ms / 1e3)
+
+    # dominant kernel: rma_decode, per-launch duration from the events around each launch
+    durs = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
+    dec_ms = sum(durs) / len(durs)
+    if kind == "batch":
+        alg_bytes = B * BYTES_FULL
+    else:
+        alg_bytes = None
+    peak, peak_kind = peaks()
+
+    # end to end through the public API: host (pinned) inputs in, host output out, every step
+    e2e = None
+    if not args.no_e2e:
+        h2d, d2h = step_input_bytes(B, L)
+        host_in = [[{k: v.cpu().pin_memory() for k, v in pool[s][l].items()} for l in range(L)] for s in range(4)]
+        host_out = torch.empty(L, B, 16, 256, dtype=torch.bfloat16).pin_memory()
+        dev_in = [{k: torch.empty_like(v, device=device) for k, v in host_in[0][l].items()} for l in range(L)]
+        outs = torch.empty(L, B, 16, 256, dtype=torch.bfloat16, device=device)
+
+        def e2e_step(i):
+            for l in range(L):
+                for k, v in host_in[i % 4][l].items():
+                    dev_in[l][k].copy_(v, non_blocking=True)
+            for l in range(L):
+                x = dev_in[l]
+                rma.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"], x["cand_score"],
+                                w[l], b[l], outs[l], ws, stream=stream)
+                rma.admit(st, l, stream=stream)
+            host_out.copy_(outs, non_blocking=True)
+
+        Ke = max(16, K // 8)
+        for i in range(3):
+            e2e_step(i)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(Ke):
+            e2e_step(i)
+        a1.record(stream)
+        torch.cuda.synchronize(device)
+        ems = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([ems], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * B * Ke / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": Ke,
+               "path": "pinned host inputs -> device copies -> rma_decode_step + rma_admit x 8 layers -> "
+                       "pinned host outputs, one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and kind == "batch":
+        try:
+            cpu = cpu_oracle_decode(n_seq=8, n_layers=8, n_steps=12)
+        except Exception as ex:   # the baseline is a report, never a reason to lose the bench line
+            cpu = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": f"failed: {ex}"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+            "config": {"workload": {"batch": "batch-512 decode: 512 sequences x 8 RMA layers, 4 KV groups x 4 "
+                                             "q-heads, head_dim 256, rings full (1023), banks full (1024), pending "
+                                             "staggered 0..255 (2 admits per layer per step)",
+                                    "long": "long-context decode: 1 sequence x 8 RMA layers, pos 131072, full ring "
+                                            "and bank, pending 0",
+                                    "ragged": f"ragged decode: {B} sequences x 8 layers, ring fill U{{1..1023}}, "
+                                              "bank fill U{0..1024}, pending U{0..255}, 16-level scores"}[kind],
+                       "batch": B, "layers": L, "step": "8 x (rma_decode_step + rma_admit)",
+                       "l2": "inputs larger than L2: the state is %.1f GB" % (st.buffer.numel() / 1e9),
+                       "parallelism": f"replicas x{world} (no data-path collective)"},
+            "gpu_launches": K * L * 2,
+            "clocks": clocks,
+            "roofline": {"bound": "hbm",
+                         "achieved": (alg_bytes / (dec_ms / 1e3) / 1e9) if alg_bytes else None,
+                         "peak": peak, "unit": "GB/s",
+                         "frac": (alg_bytes / (dec_ms / 1e3) / 1e9 / peak) if alg_bytes else None,
+                         "traffic": profiled_traffic(DECODE_PROFILE, "rma_decode.cu") if kind == "batch" else None,
+                         "kernel": "rma_decode (decode_kernel)", "kernel_ms": dec_ms,
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                         else "fallback 6.65 TB/s"},
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
