@@ -2,8 +2,9 @@
 
 Argument marshalling only: every step of decode, admit and prefill runs in
 the CUDA kernels of ``librma.so``.  PyTorch provides device memory and
-streams.  There is no CPU fallback: importing this package fails if the
-library has not been built (``python -m bounded_memory_attention_b200.build``).
+streams.  There is no CPU fallback: importing this package builds
+``librma.so`` if it is missing or older than its sources (nvcc, sm_100a) and
+fails if that is impossible.
 
 The functions mirror the C ABI in ``include/rma.h`` (same names without the
 ``rma_`` prefix); see that header for the semantics, layouts and errors.
@@ -41,8 +42,13 @@ class _Layout(ctypes.Structure):
 
 
 def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bounded_memory_attention_b200.build`")
+    from . import build as _build
+    try:
+        _build.build()          # no-op unless a source is newer than the library
+    except Exception as ex:     # no nvcc, or a compile error: there is no fallback
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing and could not be built: {ex}") from ex
+        raise ImportError(f"{LIB_PATH} is older than its sources and could not be rebuilt: {ex}") from ex
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32 = ctypes.c_void_p, ctypes.c_int
     cfgp = ctypes.POINTER(_Config)
@@ -55,6 +61,7 @@ def _load():
     lib.rma_workspace_bytes.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.rma_set_decode_splits.argtypes = [vp, i32, i32]
     lib.rma_decode_step.argtypes = [vp, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
+    lib.rma_decode_step_noalloc.argtypes = [vp, i32] + [vp] * 9 + [vp]
     lib.rma_admit.argtypes = [vp, i32, i32, vp]
     lib.rma_prefill_block.argtypes = [vp, i32, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
     lib.rma_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -63,7 +70,7 @@ def _load():
     lib.rma_last_error.argtypes = []
     lib.rma_last_error.restype = ctypes.c_char_p
     for f in ("rma_state_alloc", "rma_state_layout", "rma_workspace_bytes", "rma_set_decode_splits",
-              "rma_decode_step", "rma_admit", "rma_prefill_block", "rma_get_status"):
+              "rma_decode_step", "rma_decode_step_noalloc", "rma_admit", "rma_prefill_block", "rma_get_status"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -218,6 +225,27 @@ def decode_step(state: State, layer: int, q, k_cur, v_cur, cand_k, cand_v, cand_
         raise TypeError("ws must be a CUDA uint8 tensor")
     _check(lib.rma_decode_step(state.handle, int(layer), *args, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
                                _stream_handle(stream)), "rma_decode_step")
+    return out
+
+
+def decode_step_noalloc(state: State, layer: int, q, k_cur, v_cur, cand_k, cand_v, cand_score, w_g, b_g, out,
+                        stream=None) -> torch.Tensor:
+    """rma_decode_step_noalloc: a decode step for callers that cannot allocate device memory.
+
+    Like ``decode_step`` but without a workspace: the library's built-in 32 MiB
+    scratch per GPU holds the partials.  Calls that may overlap on the GPU
+    share that scratch and must be ordered by the caller; the first call on a
+    device should come before any stream capture.  Returns ``out``.
+    """
+    c = state.cfg
+    B, G, HQ, D = c.batch, c.n_groups, c.n_q_heads, c.head_dim
+    bf, f32 = torch.bfloat16, torch.float32
+    args = [_ptr(q, bf, B * HQ * D, "q"), _ptr(k_cur, bf, B * G * D, "k_cur"), _ptr(v_cur, bf, B * G * D, "v_cur"),
+            _ptr(cand_k, bf, B * G * D, "cand_k"), _ptr(cand_v, bf, B * G * D, "cand_v"),
+            _ptr(cand_score, f32, B * G, "cand_score"), _ptr(w_g, f32, HQ * D, "w_g"), _ptr(b_g, f32, HQ, "b_g"),
+            _ptr(out, bf, B * HQ * D, "out")]
+    _check(lib.rma_decode_step_noalloc(state.handle, int(layer), *args, _stream_handle(stream)),
+           "rma_decode_step_noalloc")
     return out
 
 

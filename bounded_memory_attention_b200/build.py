@@ -1,6 +1,7 @@
 """Build librma.so in-tree with nvcc for sm_100a.
 
-Usage: python -m bounded_memory_attention_b200.build   (or build() from Python)
+Usage: python -m bounded_memory_attention_b200.build [--force] [--ptxas-v]
+Importing the package runs build() too (a no-op when the library is fresh).
 """
 from __future__ import annotations
 
@@ -38,11 +39,12 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if not force and not _stale():
         return LIB
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    cmd = [NVCC, *FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-shared", "-o", LIB + ".tmp", *srcs]
+    tmp = f"{LIB}.{os.getpid()}.tmp"
+    cmd = [NVCC, *FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp, *srcs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 

@@ -253,6 +253,29 @@ int rma_decode_step(rma_state* st, int layer, const uint16_t* q, const uint16_t*
     return RMA_OK;
 }
 
+int rma_decode_step_noalloc(rma_state* st, int layer, const uint16_t* q, const uint16_t* k_cur,
+                            const uint16_t* v_cur, const uint16_t* cand_k, const uint16_t* cand_v,
+                            const float* cand_score, const float* w_g, const float* b_g, uint16_t* out,
+                            void* stream) {
+    State* s = as_state(st);
+    int rc = check_layer(s, layer);
+    if (rc != RMA_OK) return rc;
+    const Splits sp = decode_splits(*s);
+    const size_t need =
+        (size_t)s->cfg.batch * s->cfg.n_groups * (sp.ring_splits + sp.bank_splits) * kPartialFloats * 4;
+    if (need > kStaticDecodeScratchBytes)
+        return fail(RMA_ERR_BUFFER_TOO_SMALL,
+                    "rma_decode_step_noalloc: this batch and split shape need " + std::to_string(need) +
+                        " bytes of scratch but the built-in scratch holds " +
+                        std::to_string(kStaticDecodeScratchBytes) +
+                        " (use fewer sequences per call, fewer splits, or rma_decode_step with a workspace)");
+    void* scratch = nullptr;
+    cudaError_t e = static_decode_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "looking up the built-in decode scratch");
+    return rma_decode_step(st, layer, q, k_cur, v_cur, cand_k, cand_v, cand_score, w_g, b_g, out, scratch,
+                           kStaticDecodeScratchBytes, stream);
+}
+
 int rma_admit(rma_state* st, int layer, int force, void* stream) {
     State* s = as_state(st);
     int rc = check_layer(s, layer);

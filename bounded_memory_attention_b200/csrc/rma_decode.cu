@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "rma_internal.cuh"
 
 namespace rma {
@@ -453,5 +455,34 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 int decode_max_splits() { return kMaxSplits; }
+
+// ---------------------------------------------------------------------------
+// Built-in decode scratch, for callers that cannot allocate device memory.
+// A fixed 32 MiB array in the library's device image: every GPU that loads
+// the library holds it until the process exits.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in symbol); its
+// device address is looked up once per device with cudaGetSymbolAddress,
+// with that device current, and cached.  All calls on a device share it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticDecodeScratchBytes];
+
+cudaError_t static_decode_scratch(void** ptr) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
 
 }  // namespace rma

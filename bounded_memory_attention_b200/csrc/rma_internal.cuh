@@ -76,6 +76,11 @@ struct PrefillArgs {
 // m[4] (running max, log2 domain), l[4] (sum of exponentials), acc[4][D].
 constexpr int kPartialFloats = 4 + 4 + kQPerGroup * kHeadDim;
 
+// Size of the library's own decode scratch (rma_decode_step_noalloc).
+constexpr size_t kStaticDecodeScratchBytes = size_t(32) << 20;
+// Device address of that scratch on the current device (set up on first use per device).
+cudaError_t static_decode_scratch(void** ptr);
+
 // Launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream);

@@ -163,6 +163,31 @@ RMA_API int rma_decode_step(rma_state* st, int layer,
                     const float* w_g, const float* b_g, uint16_t* out,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* rma_decode_step without a caller-supplied workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory when they call: for example a plug-in inside a host
+ * framework that owns all device memory and hands out no scratch, a
+ * real-time serving loop that forbids allocation after start-up, or an
+ * embedded deployment that reserves its memory once.  Such a caller still
+ * passes its inputs and outputs; the per-split partials go to a scratch
+ * array built into the library (32 MiB per GPU, held on every GPU that loads
+ * the library until the process exits).  The call allocates nothing.
+ *   Limit: batch * n_groups * (ring_splits + bank_splits) * 4128 bytes must
+ *   fit in 32 MiB (batch 512 with the default split shape needs 16.9 MB);
+ *   larger calls return RMA_ERR_BUFFER_TOO_SMALL and launch nothing.
+ *   The first call on each device looks up the scratch's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   One scratch per GPU is shared by every call on it, and keeps whatever the
+ *   last call left: calls that can overlap on the GPU (other streams, other
+ *   states) race on it, so the caller must order them.  Nothing in it needs to
+ *   start at zero: each partial is written before it is read.
+ * Arguments, alignment and results are those of rma_decode_step. */
+RMA_API int rma_decode_step_noalloc(rma_state* st, int layer,
+                                    const uint16_t* q, const uint16_t* k_cur, const uint16_t* v_cur,
+                                    const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
+                                    const float* w_g, const float* b_g, uint16_t* out, void* stream);
+
 /* Admit at RMA layer `layer` ([NEWS] "How it works": after every 256
  * candidates the existing anchors and the candidates compete and the top
  * 1,024 are kept, independently per KV group; [SITE] "Commit interval 256").
