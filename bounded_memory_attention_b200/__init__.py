@@ -24,6 +24,7 @@ STATUS_PENDING_OVERFLOW = 1
 STATUS_NAN_SCORE = 2
 STATUS_PREFILL_PENDING_OVERFLOW = 4
 STATUS_BAD_COUNTERS = 8
+STATUS_TIMEOUT = 16
 
 ERRORS = {0: "RMA_OK", -1: "RMA_ERR_INVALID_ARG", -2: "RMA_ERR_UNSUPPORTED", -3: "RMA_ERR_BUFFER_TOO_SMALL",
           -4: "RMA_ERR_CUDA", -5: "RMA_ERR_MISALIGNED"}

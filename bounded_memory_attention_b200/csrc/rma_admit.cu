@@ -71,7 +71,11 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
     return r;
 }
 
-__global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__ LayerView s, int force) {
+// prefill_n > 0: first account for a prefill block of prefill_n tokens whose
+// K/V and candidates were already written (pos += n; pend_fill += n if the
+// candidates fit, else RMA_STATUS_PREFILL_PENDING_OVERFLOW).
+__global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__ LayerView s, int force,
+                                                         int prefill_n) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int g = blockIdx.x, b = blockIdx.y;
     const int bg = b * s.G + g;
@@ -83,6 +87,16 @@ __global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__
         if (threadIdx.x == 0) atomicOr(s.status, (unsigned)RMA_STATUS_BAD_COUNTERS);
         nb = min(max(nb, 0), s.A);
         np = min(max(np, 0), s.P);
+    }
+    if (prefill_n > 0) {
+        const bool fits = np + prefill_n <= s.P;
+        __syncthreads();   // every thread has read the counters
+        if (tid == 0) {
+            cnt[0] = max(cnt[0], 0) + prefill_n;
+            if (fits) cnt[2] = np + prefill_n;
+            else atomicOr(s.status, (unsigned)RMA_STATUS_PREFILL_PENDING_OVERFLOW);
+        }
+        if (fits) np += prefill_n;
     }
     if (!(np == s.P || (force && np > 0))) return;
 
@@ -212,7 +226,7 @@ size_t admit_smem_bytes(int A, int P) {
     return off + (size_t)(2 * P + 32) * 4;
 }
 
-cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream) {
+cudaError_t launch_admit(const LayerView& s, int force, int prefill_n, cudaStream_t stream) {
     const size_t smem = admit_smem_bytes(s.A, s.P);
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
@@ -221,7 +235,7 @@ cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream) {
         configured = smem;
     }
     dim3 grid(s.G, s.B);
-    admit_kernel<<<grid, kThreads, smem, stream>>>(s, force);
+    admit_kernel<<<grid, kThreads, smem, stream>>>(s, force, prefill_n);
     return cudaGetLastError();
 }
 

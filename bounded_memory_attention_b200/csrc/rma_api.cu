@@ -281,7 +281,7 @@ int rma_admit(rma_state* st, int layer, int force, void* stream) {
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;
     if (force != 0 && force != 1) return fail(RMA_ERR_INVALID_ARG, "force must be 0 or 1");
-    cudaError_t e = launch_admit(layer_view(*s, layer), force, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_admit(layer_view(*s, layer), force, 0, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_admit");
     return RMA_OK;
 }
@@ -320,7 +320,7 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
     cudaError_t e = launch_prefill(a, cs);
     if (e == cudaErrorNotSupported) return fail(RMA_ERR_UNSUPPORTED, "rma_prefill_block is not available in this build");
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_prefill_block");
-    e = launch_admit(a.s, 1, cs);
+    e = launch_admit(a.s, 1, n_tok, cs);
     if (e != cudaSuccess) return cuda_fail(e, "launching the forced admit");
     return RMA_OK;
 }

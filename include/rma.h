@@ -71,6 +71,10 @@ extern "C" {
  * [0, bank_slots], pend_fill not in [0, pend_slots]), e.g. a corrupted restore:
  * it clamped them for its own indexing and went on. */
 #define RMA_STATUS_BAD_COUNTERS              8u
+/* A kernel gave up waiting on one of its own pipeline barriers (a bounded
+ * wait of about two seconds ran out) and abandoned its tile; its outputs are
+ * not valid.  Indicates a fault in the library, never an input condition. */
+#define RMA_STATUS_TIMEOUT                  16u
 
 /* Dimensions.  This build implements q_per_group == 4 and head_dim == 256
  * (RMA_ERR_UNSUPPORTED otherwise), any n_groups >= 1, ring_slots in

@@ -1,0 +1,124 @@
+"""GPU parity: rma_prefill_block (tcgen05 attention, commit, forced admit) against the oracle.
+
+Outputs within 1e-2 max(1, |oracle|) element by element; the whole state
+(ring, bank, scores, pending, counters) bit-exact after every block.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+from _gpu import TOL, assert_state_equal, gpu_state_np, lib, make_pair, output_error
+from _util import to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _block_both(rma, st, ost, layer, seed, w, b, ws, quantized=False):
+    cfg = st.cfg
+    n = cfg.pend_slots
+    x = si.prefill_inputs(cfg.batch, n, cfg.n_groups, cfg.q_per_group, cfg.head_dim, seed=seed,
+                          quantized_scores=quantized)
+    xd = {k: v.cuda() for k, v in x.items()}
+    out = torch.empty(cfg.batch, n, cfg.n_groups * cfg.q_per_group, cfg.head_dim, dtype=torch.bfloat16,
+                      device="cuda")
+    rma.prefill_block(st, layer, xd["q"], xd["k"], xd["v"], xd["cand_k"], xd["cand_v"], xd["cand_score"],
+                      w, b, out, ws)
+    xn = {k: to_np(v) for k, v in x.items()}
+    ref = oracle.prefill_block(ost, layer, xn["q"], xn["k"], xn["v"], xn["cand_k"], xn["cand_v"],
+                               xn["cand_score"], to_np(w), to_np(b))
+    torch.cuda.synchronize()
+    return to_np(out), ref
+
+
+def test_prefill_from_empty_state_five_blocks():
+    """Blocks at s = 0, 256, 512, 768, 1024: empty, partial, full and wrapped rings; the bank fills by admits."""
+    rma = lib()
+    cfg = oracle.Config(batch=2, n_layers=1)
+    st, ost = make_pair(cfg, seed=21, **si.workload_counters("empty", 1, 2, 4))
+    w, b = si.gate_params(1, 16, 256, seed=21)
+    w, b = w[0].cuda(), si.f32_normal((16,), 22, std=0.5).cuda()
+    ws = st.workspace(256)
+    for blk in range(5):
+        g_out, ref = _block_both(rma, st, ost, 0, 500 + blk, w, b, ws)
+        err = output_error(g_out, ref)
+        assert err <= TOL, f"block {blk}: output error {err}"
+        assert_state_equal(gpu_state_np(st), ost, f"block {blk}")
+        assert rma.get_status(st) == 0, f"block {blk}"
+
+
+def test_prefill_on_long_history_with_quantized_scores():
+    """Ring full at an arbitrary rotation (pos = 131,089), bank full, ties in the admit."""
+    rma = lib()
+    cfg = oracle.Config(batch=3, n_layers=2)
+    st, ost = make_pair(cfg, seed=23, pos=131_089, bank_fill=1024, pend_fill=0, quantized=True)
+    w, b = si.gate_params(2, 16, 256, seed=23)
+    w, b = w.cuda(), b.cuda()
+    ws = st.workspace(256)
+    for blk in range(3):
+        for layer in (1, 0):
+            g_out, ref = _block_both(rma, st, ost, layer, 600 + 2 * blk + layer, w[layer], b[layer], ws,
+                                     quantized=True)
+            err = output_error(g_out, ref)
+            assert err <= TOL, f"block {blk} layer {layer}: output error {err}"
+        assert_state_equal(gpu_state_np(st), ost, f"block {blk}")
+
+
+def test_prefill_partial_bank_and_small_block():
+    """P = 64 (two tiles per block), bank partly filled, ring partly filled."""
+    rma = lib()
+    cfg = oracle.Config(batch=2, n_layers=1, pend_slots=64, bank_slots=300, ring_slots=200)
+    st, ost = make_pair(cfg, seed=25, pos=[[[70] * 4, [450] * 4]], bank_fill=[[[0] * 4, [137] * 4]],
+                        pend_fill=0)
+    w, b = si.gate_params(1, 16, 256, seed=25, std=0.2)
+    w, b = w[0].cuda(), si.f32_normal((16,), 26, std=0.5).cuda()
+    ws = st.workspace(64)
+    for blk in range(6):
+        g_out, ref = _block_both(rma, st, ost, 0, 700 + blk, w, b, ws)
+        err = output_error(g_out, ref)
+        assert err <= TOL, f"block {blk}: output error {err}"
+        assert_state_equal(gpu_state_np(st), ost, f"block {blk}")
+
+
+def test_prefill_candidates_that_do_not_fit_are_flagged():
+    rma = lib()
+    cfg = oracle.Config(batch=1, n_layers=1)
+    st, ost = make_pair(cfg, seed=27, pos=5000, bank_fill=1000, pend_fill=3)
+    w, b = si.gate_params(1, 16, 256, seed=27)
+    w, b = w[0].cuda(), b[0].cuda()
+    g_out, ref = _block_both(rma, st, ost, 0, 800, w, b, st.workspace(256))
+    assert output_error(g_out, ref) <= TOL
+    assert_state_equal(gpu_state_np(st), ost, "overflow block")
+    assert rma.get_status(st) == rma.STATUS_PREFILL_PENDING_OVERFLOW
+    assert ost.status == oracle.STATUS_PREFILL_PENDING_OVERFLOW
+
+
+def test_prefill_then_decode_handoff():
+    """A prefill block leaves pending empty; decode steps continue from it with the oracle in step."""
+    rma = lib()
+    cfg = oracle.Config(batch=2, n_layers=1)
+    st, ost = make_pair(cfg, seed=29, pos=700, bank_fill=512, pend_fill=0)
+    w, b = si.gate_params(1, 16, 256, seed=29)
+    w, b = w[0].cuda(), b[0].cuda()
+    g_out, ref = _block_both(rma, st, ost, 0, 900, w, b, st.workspace(256))
+    assert output_error(g_out, ref) <= TOL
+    ws1 = st.workspace(1)
+    out = torch.empty(2, 16, 256, dtype=torch.bfloat16, device="cuda")
+    for t in range(5):
+        x = {k: v.cuda() for k, v in si.decode_inputs(2, 4, 4, 256, seed=950 + t).items()}
+        rma.decode_step(st, 0, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"], x["cand_score"],
+                        w, b, out, ws1)
+        rma.admit(st, 0)
+        xn = {k: to_np(v) for k, v in x.items()}
+        r = oracle.decode_step(ost, 0, xn["q"], xn["k_cur"], xn["v_cur"], xn["cand_k"], xn["cand_v"],
+                               xn["cand_score"], to_np(w), to_np(b))
+        oracle.admit(ost, 0)
+        assert output_error(to_np(out), r) <= TOL
+    assert_state_equal(gpu_state_np(st), ost, "after handoff")
