@@ -21,12 +21,14 @@
 //   packed FFMA2.  Warps merge in shared memory into one (m, l, acc) partial
 //   per CTA; the last CTA of (b, g) to arrive (atomic ticket, no waiting)
 //   merges all partials, adds the current token and the gate, writes the
-//   output and performs the state writes after every read of the step.
+//   output and performs the state writes after every read of the step; when
+//   the step fills the pending buffer it also runs the admit for (b, g).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
 #include <mutex>
 
+#include "rma_admit_impl.cuh"
 #include "rma_internal.cuh"
 
 namespace rma {
@@ -44,6 +46,7 @@ constexpr int kSmemBytes = kPipeBytes + kWarps * kBcastFloats * 4 + (kMaxSplits 
 
 static_assert(kWarps == 8, "merger assigns 8 dot products to 8 warps");
 static_assert(kStages * kStageBytes >= kPartialFloats * 4, "per-warp pipeline region must hold one warp partial");
+static_assert(kPipeBytes >= admit_scratch_bytes(1, 4095), "the admit reuses the pipeline region (any A + P <= 4096)");
 
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -436,6 +439,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         c[0] = pos + 1;
         c[2] = room ? pend_fill + 1 : pend_fill;
         a.s.tickets[bg] = 0u;
+    }
+
+    // ---- the admit, in this launch, when this step filled the pending buffer ----
+    // Every split of (b, g) has finished reading the bank, so the bank may change now.
+    if (room && pend_fill + 1 == a.s.P) {
+        __syncthreads();   // the appended candidate and counters are visible to the whole CTA
+        admit_group<kThreads>(a.s, bg, bank_fill, a.s.P, smem);
     }
 }
 

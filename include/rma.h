@@ -159,8 +159,12 @@ RMA_API int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_split
  *   b_g        f32  [n_groups*q_per_group]
  *   out        bf16 [batch][n_groups*q_per_group][head_dim]   (written)
  *   ws         workspace of rma_workspace_bytes(st, 1) bytes
+ * When this step fills a group's pending buffer (pend_fill reaches P), the
+ * admit of that (sequence, group) runs in the same launch, after every read
+ * of the step, exactly as rma_admit would (so calling rma_admit afterwards
+ * finds nothing to do); its records are visible from the next step on.
  * All pointers are device pointers; q, k_cur, v_cur, cand_k, cand_v, w_g and
- * out must be 16-byte aligned.  Does not run the admit: call rma_admit next. */
+ * out must be 16-byte aligned. */
 RMA_API int rma_decode_step(rma_state* st, int layer,
                     const uint16_t* q, const uint16_t* k_cur, const uint16_t* v_cur,
                     const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
@@ -224,9 +228,10 @@ RMA_API int rma_admit(rma_state* st, int layer, int force, void* stream);
  *   w_g, b_g    as in rma_decode_step
  *   out         bf16 [batch][n_tok][n_groups*q_per_group][head_dim]  (written)
  *   ws          workspace of rma_workspace_bytes(st, n_tok) bytes
- * This build requires n_tok == pend_slots, n_tok a multiple of 32 and
- * n_tok <= ring_slots (RMA_ERR_UNSUPPORTED otherwise).  Alignment as in
- * rma_decode_step. */
+ * One launch: the admit runs inside it once every read of the block is done.
+ * This build requires n_tok == pend_slots, n_tok a multiple of 32, at most
+ * 256 and at most ring_slots (RMA_ERR_UNSUPPORTED otherwise).  Alignment as
+ * in rma_decode_step. */
 RMA_API int rma_prefill_block(rma_state* st, int layer, int n_tok,
                       const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
