@@ -298,9 +298,9 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
     for (const void* p : a16)
         if (!aligned(p, 16)) return fail(RMA_ERR_MISALIGNED, "q, k, v, cand_k, cand_v, w_g, out, ws need 16-byte alignment");
     if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
-    if (n_tok != s->cfg.pend_slots || n_tok % 32 != 0 || n_tok > 256 || n_tok > s->cfg.ring_slots)
+    if (n_tok != s->cfg.pend_slots || n_tok % 64 != 0 || n_tok > 256 || n_tok > s->cfg.ring_slots)
         return fail(RMA_ERR_UNSUPPORTED,
-                    "this build needs n_tok == pend_slots, a multiple of 32, at most 256 and at most ring_slots");
+                    "this build needs n_tok == pend_slots, a multiple of 64, at most 256 and at most ring_slots");
     if (ws_bytes < prefill_workspace_bytes(s->cfg, n_tok))
         return fail(RMA_ERR_BUFFER_TOO_SMALL, "workspace smaller than rma_workspace_bytes(st, n_tok)");
     PrefillArgs a;

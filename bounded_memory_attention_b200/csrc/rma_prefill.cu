@@ -10,31 +10,38 @@
 // Then the block's K/V go into the ring, its candidates into pending, and
 // the admit runs forced.
 //
-// One launch.  One CTA per (sequence, group, tile of 32 tokens, phase):
-// phase 0 reads the local window, phase 1 the bank.  The tile's 128 rows are
-// 32 tokens x the group's 4 query heads, which share every key, so one K/V
-// chunk feeds all 4 heads.
-//   * tensor memory (512 columns): O [0,256) FP32, S/P double buffer
-//     [256,320) and [320,384), Q [384,512) as packed BF16 (the A operand of
-//     Q K^T comes from tensor memory, which leaves shared memory to a
-//     three-stage ring of 64-key K/V chunks);
-//   * warp 8 (TMA) loads 128B-swizzled K and V chunks: ring slots, then the
-//     block's own keys, or bank slots;
-//   * warp 9 issues tcgen05.mma: S = Q K^T (M 128, N 64, K 256) and
-//     O += P V (M 128, N 256, K 64; P from tensor memory, V an MN-major
-//     shared-memory operand);
-//   * warps 0-7 are the softmax: two warpgroups, each thread one row and one
-//     half of the chunk's keys (and of Q and O's columns).  They load Q into
-//     tensor memory, then per chunk read their half of S, mask it by
-//     position (whole halves that are all visible or all hidden skip the
-//     per-key test), exchange the row max through shared memory, keep the
-//     online max / sum in FP32 (moving the reference max only when it grows by
-//     more than 2^8), write BF16 P over S, and finally normalise O.
-// Tail, through a per-(sequence, group) ticket word: each CTA writes its
-// normalised rows to the workspace; the second CTA of a tile's pair adds
-// them as local + gate * anchor and writes the BF16 output; the last CTA of
-// the (sequence, group) writes the block into the ring and pending buffer
-// (every read of the block is finished by then) and runs the forced admit.
+// One launch.  A CTA owns 128 query rows (32 tokens x the group's 4 query
+// heads, which share every key) and one phase: the local window (phase 0) or
+// the bank (phase 1).  Four CTAs form a thread-block cluster:
+//   rank 0: tile 2p, local     rank 1: tile 2p+1, local
+//   rank 2: tile 2p, anchor    rank 3: tile 2p+1, anchor
+// Ranks (0,1) and (2,3) are CTA pairs for the 2-SM tensor-core MMA
+// (tcgen05 cta_group::2, M = 256): both tiles of a pair read exactly the same
+// keys, so each CTA loads only half of every 64-key K/V chunk (K rows split
+// by key, V split by dimension), which halves the K/V bytes per FLOP.
+//   * tensor memory (512 columns, the pair allocates together): O [0,256)
+//     FP32, S/P double buffer [256,320) and [320,384), Q [384,512) packed
+//     BF16 (Q K^T takes A from tensor memory; shared memory holds a six-stage
+//     ring of K/V half-chunks);
+//   * warp 8 of each CTA loads its half of each chunk with TMA (128B swizzle);
+//   * warp 9 of the even CTA issues S = Q K^T (N 64, K 256) and O += P V
+//     (N 256, K 64, P from tensor memory, V an MN-major operand) and commits
+//     to the barriers of both CTAs; warp 9 of the odd CTA checks its half
+//     landed, clears stale V rows and signals the even CTA;
+//   * warps 0-7 of each CTA are the softmax for its own rows: two
+//     warpgroups, each thread one row and half of the chunk's keys; they load
+//     Q into tensor memory, read S, mask by position (whole halves that are
+//     all visible or all hidden skip the per-key test), exchange the row max
+//     through shared memory, keep the online max / sum in FP32 (moving the
+//     reference max only when it grows by more than 2^8), write BF16 P over
+//     S, and finally normalise O.
+// Tail: every CTA writes its normalised rows into its own shared memory; after
+// a cluster barrier the local and anchor CTAs of a tile each combine half of
+// its rows, reading the other result through distributed shared memory:
+// out = local + gate * anchor in FP32, rounded once to BF16.  A per-(sequence,
+// group) ticket finds the last CTA, which writes the block into the ring and
+// the pending buffer (every read of the block is over by then) and runs the
+// forced admit.  No load is multicast: every CTA reads its own data.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -49,39 +56,47 @@
 namespace rma {
 namespace {
 
-constexpr int kTileTok = 32;                          // tokens per tile
-constexpr int kRows = kTileTok * kQPerGroup;          // 128 MMA rows
+constexpr int kTileTok = 32;                          // tokens per CTA
+constexpr int kRows = kTileTok * kQPerGroup;          // 128 rows per CTA, 256 per pair
 constexpr int kChunk = 64;                            // keys per chunk
-constexpr int kMaxTiles = 8;                          // ticket word: 2 bits per tile below bit 16
-constexpr int kSlabKV = kChunk * 128;                 // 64 keys x 64 dims (bf16) = 8 KiB
-constexpr int kKVBytes = 4 * kSlabKV;                 // 32 KiB per K or V chunk
-constexpr int kStages = 3;
-constexpr int kSmemK = 0;
-constexpr int kSmemV = kStages * kKVBytes;
-constexpr int kSmemBar = 2 * kStages * kKVBytes;      // 192 KiB
-constexpr int kSmemXch = kSmemBar + 256;             // softmax exchange: max [2][2][128], sums/gate [2][128]
+constexpr int kHalfKeys = kChunk / 2;                 // K rows each CTA of a pair loads
+constexpr int kSlabK = kHalfKeys * 128;               // 32 keys x 64 dims (bf16) = 4 KiB
+constexpr int kSlabV = kChunk * 128;                  // 64 keys x 64 dims = 8 KiB
+constexpr int kKHalfBytes = 4 * kSlabK;               // 16 KiB: this CTA's keys, all 256 dims
+constexpr int kVHalfBytes = 2 * kSlabV;               // 16 KiB: all 64 keys, this CTA's 128 dims
+constexpr int kStageBytes = kKHalfBytes + kVHalfBytes;
+constexpr int kStages = 6;
+constexpr int kSmemBar = kStages * kStageBytes;       // 192 KiB
+// softmax exchange (floats): the reference max handed between the groups [128] at 0, each
+// group's final reference max [2][128] at 128 and row sum [2][128] at 512, the gate [128] at 768
+// (first the two halves' partial dot products [2][128], then the gate itself in the first)
+constexpr int kSmemXch = kSmemBar + 512;
 constexpr int kSmemBytes = kSmemXch + 4096 + 1024;    // + 1 KiB for alignment
+constexpr int kXchEndM = 128, kXchEndL = 512, kXchGate = 768;
 constexpr int kSoftmaxThreads = 256;                  // warps 0-7
 constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
+constexpr int kTilesPerCluster = 2;
 
+static_assert(kSmemBar >= kRows * 1024, "the result rows reuse the K/V stages");
 static_assert(kSmemBar >= (int)admit_scratch_bytes(1, 4095), "the tail's admit reuses the K/V stages");
 
 struct Tmaps {
-    CUtensorMap k, v, ring_k, ring_v, bank_k, bank_v;
+    CUtensorMap k, v, ring_k, ring_v, bank_k, bank_v;   // K maps: 32-row boxes; V maps: 64-row boxes
 };
 
 enum Bar {
-    kQReady = 0,
-    kKFull = 1,                 // [3]
-    kVFull = 4,                 // [3]
-    kKVEmpty = 7,               // [3]
-    kSFull = 10,                // [2]
-    kPFull = 12,                // [2]
-    kODone = 14,
-    kNumBars = 15
+    kQReady = 0,                // even CTA: 16 arrivals (8 warps x 2 CTAs)
+    kFull = 1,                  // [6] even CTA: own loads (tx) + the odd CTA's signal; odd CTA: own loads
+    kEmpty = 7,                 // [6] both: the MMA commit after P V of the chunk in that stage
+    kSFull = 13,                // [2] both: MMA commit after Q K^T
+    kPFull = 15,                // [2] even CTA, one per softmax group: 8 arrivals (4 warps x 2 CTAs)
+    kODone = 17,                // both: MMA commit after P V
+    kXfer = 18,                 // both: the other CTA's half-result rows have landed (tx bytes)
+    kOFinal = 19,               // both: MMA commit after the last P V (one phase)
+    kNumBars = 20
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -95,16 +110,21 @@ __device__ __forceinline__ float fast_ex2(float x) {
     return y;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ Tmaps tm, const __grid_constant__ PrefillArgs a, int ntiles) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const LayerView& S = a.s;
-    const int T = blockIdx.x >> 1, phase = blockIdx.x & 1;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int pr = rank & 1;                     // 0: the pair's MMA-issuing CTA
+    const int phase = rank >> 1;
+    const int T = kTilesPerCluster * (blockIdx.x >> 2) + pr;
     const int g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = S.G, HQ = G * kQPerGroup, n = a.n_tok;
     const int bg = b * G + g;
+    const uint32_t leader = rank & ~1u;
+    const uint16_t pair_mask = (uint16_t)(3u << leader);
 
     const int32_t* cnt = S.counters + bg * 4;
     const int s = max(cnt[0], 0);
@@ -112,154 +132,175 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pend_fill = min(max(cnt[2], 0), S.P);
     const int fill = min(s, S.R);
 
+    // chunks (identical for both CTAs of a pair: tiles 2p and 2p+1 need block chunks 0..p)
     int n_ring = 0, n_blk = 0, n_bank = 0;
     if (phase == 0) {
         n_ring = (fill + kChunk - 1) / kChunk;
-        n_blk = (kTileTok * T + kTileTok - 1) / kChunk + 1;
+        n_blk = (kTileTok * (T | 1) + kTileTok - 1) / kChunk + 1;
     } else {
         n_bank = (bank_fill + kChunk - 1) / kChunk;
     }
     const int nchunks = n_ring + n_blk + n_bank;
-    const bool has_work = nchunks > 0;
-    float* own_rows = a.ws + (((size_t)bg * ntiles + T) * 2 + phase) * (size_t)kRows * kHeadDim;
-    const float* partner_rows = a.ws + (((size_t)bg * ntiles + T) * 2 + (phase ^ 1)) * (size_t)kRows * kHeadDim;
+    const bool has_work = nchunks > 0;        // uniform over the pair
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars + 1);
-    int* tail_flags = reinterpret_cast<int*>(bars + kNumBars + 2);   // [0] partner done, [1] last of all
+    int* tail_flag = reinterpret_cast<int*>(bars + kNumBars + 2);
 
-    // softmax-thread identity (warps 0-7): row, and which half of keys / columns
-    const int row = 32 * (warp & 3) + lane;
-    const int wg = (warp >> 2) & 1;
-    const int tok = kTileTok * T + (row >> 2);    // token within the block
+    const int row = 32 * (warp & 3) + lane;   // softmax threads: row of this CTA
+    const int wg = (warp >> 2) & 1;           // and which half of keys / columns
+    const int tok = kTileTok * T + (row >> 2);
     const int head = g * kQPerGroup + (row & 3);
     float* xch = reinterpret_cast<float*>(smem + kSmemXch);
     float l = 0.f;
     uint32_t tmem = 0;
 
-    if (has_work) {
-        if (tid == 0) {
-            ptx::mbar_init(&bars[kQReady], 8);
-            for (int i = 0; i < kStages; ++i) {
-                ptx::mbar_init(&bars[kKFull + i], 1);
-                ptx::mbar_init(&bars[kVFull + i], 1);
-                ptx::mbar_init(&bars[kKVEmpty + i], 1);
-            }
-            for (int i = 0; i < 2; ++i) {
-                ptx::mbar_init(&bars[kSFull + i], 1);
-                ptx::mbar_init(&bars[kPFull + i], 8);
-            }
-            ptx::mbar_init(&bars[kODone], 1);
-            *abort_flag = 0;
-            ptx::fence_mbar_init();
+    if (tid == 0) {
+        ptx::mbar_init(&bars[kQReady], 16);
+        for (int i = 0; i < kStages; ++i) {
+            ptx::mbar_init(&bars[kFull + i], pr == 0 ? 2 : 1);
+            ptx::mbar_init(&bars[kEmpty + i], 1);
         }
-        if (warp == kWarpMma) {
-            ptx::tmem_alloc(tmem_holder, kTmemCols);
-            ptx::tmem_relinquish();
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&bars[kSFull + i], 1);
+            ptx::mbar_init(&bars[kPFull + i], 8);
         }
-        ptx::tc_fence_before();
-        __syncthreads();
-        ptx::tc_fence_after();
-        tmem = *tmem_holder;
+        ptx::mbar_init(&bars[kODone], 1);
+        ptx::mbar_init(&bars[kXfer], 1);
+        ptx::mbar_init(&bars[kOFinal], 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (has_work && warp == kWarpMma) {
+        ptx::tmem_alloc2(tmem_holder, kTmemCols);
+        ptx::tmem_relinquish2();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();   // barriers of all four CTAs initialised, tensor memory allocated
+    ptx::tc_fence_after();
+    if (has_work) tmem = *tmem_holder;
 
+    // number of valid keys of chunk j (rows past it may hold stale bytes)
+    auto chunk_valid = [&](int j) -> int {
+        if (j < n_ring) return fill - kChunk * j;
+        if (j < n_ring + n_blk) return n - kChunk * (j - n_ring);
+        return bank_fill - kChunk * (j - n_ring - n_blk);
+    };
+    // clear V rows [nvalid, 64) of this CTA's half in stage st so that P = 0 times V stays 0
+    auto clear_stale_v = [&](int j, int st) {
+        const int nvalid = chunk_valid(j);
+        if (nvalid < kChunk) {
+            uint8_t* vst = smem + st * kStageBytes + kKHalfBytes;
+            const int nz = (kChunk - nvalid) * 8;   // 16-byte pieces per slab
+            for (int e = lane; e < 2 * nz; e += 32) {
+                const int slab = e / nz, piece = e % nz;
+                reinterpret_cast<uint4*>(vst + slab * kSlabV + nvalid * 128)[piece] = make_uint4(0, 0, 0, 0);
+            }
+            ptx::fence_proxy_async_smem();
+        }
+        __syncwarp();
+    };
+
+    if (has_work) {
         if (warp == kWarpTma) {
-            // ---------------- TMA producer (whole warp loops; lane 0 issues) ----------------
+            // ---------------- TMA producer: this CTA's half of every chunk ----------------
             const int zreg = b * G + g;
             for (int j = 0; j < nchunks; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages &&
-                    !ptx::mbar_wait_warp(&bars[kKVEmpty + st], ((j / kStages) - 1) & 1, abort_flag, S.status))
+                    !ptx::mbar_wait_warp(&bars[kEmpty + st], ((j / kStages) - 1) & 1, abort_flag, S.status))
                     break;
                 if (lane == 0) {
                     const CUtensorMap* mk;
                     const CUtensorMap* mv;
-                    int y, z;
+                    int yk, zk, yv, zv;
                     if (j < n_ring) {
-                        mk = &tm.ring_k; mv = &tm.ring_v; y = kChunk * j; z = zreg;
+                        mk = &tm.ring_k; mv = &tm.ring_v;
+                        yk = kChunk * j + kHalfKeys * pr; zk = zreg; yv = kChunk * j; zv = zreg;
                     } else if (j < n_ring + n_blk) {
-                        mk = &tm.k; mv = &tm.v; y = g; z = b * n + kChunk * (j - n_ring);
+                        const int t0 = b * n + kChunk * (j - n_ring);
+                        mk = &tm.k; mv = &tm.v;
+                        yk = g; zk = t0 + kHalfKeys * pr; yv = g; zv = t0;
                     } else {
-                        mk = &tm.bank_k; mv = &tm.bank_v; y = kChunk * (j - n_ring - n_blk); z = zreg;
+                        const int a0 = kChunk * (j - n_ring - n_blk);
+                        mk = &tm.bank_k; mv = &tm.bank_v;
+                        yk = a0 + kHalfKeys * pr; zk = zreg; yv = a0; zv = zreg;
                     }
-                    ptx::mbar_arrive_expect_tx(&bars[kKFull + st], kKVBytes);
+                    uint8_t* stage = smem + st * kStageBytes;
+                    ptx::mbar_arrive_expect_tx(&bars[kFull + st], kStageBytes);
                     for (int slab = 0; slab < 4; ++slab)
-                        ptx::tma_load_3d(smem + kSmemK + st * kKVBytes + slab * kSlabKV, mk, &bars[kKFull + st],
-                                         64 * slab, y, z);
-                    ptx::mbar_arrive_expect_tx(&bars[kVFull + st], kKVBytes);
-                    for (int slab = 0; slab < 4; ++slab)
-                        ptx::tma_load_3d(smem + kSmemV + st * kKVBytes + slab * kSlabKV, mv, &bars[kVFull + st],
-                                         64 * slab, y, z);
+                        ptx::tma_load_3d(stage + slab * kSlabK, mk, &bars[kFull + st], 64 * slab, yk, zk);
+                    for (int slab = 0; slab < 2; ++slab)
+                        ptx::tma_load_3d(stage + kKHalfBytes + slab * kSlabV, mv, &bars[kFull + st],
+                                         128 * pr + 64 * slab, yv, zv);
                 }
                 __syncwarp();
             }
+        } else if (warp == kWarpMma && pr == 1) {
+            // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
+            for (int j = 0; j < nchunks; ++j) {
+                const int st = j % kStages;
+                if (!ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
+                clear_stale_v(j, st);
+                if (lane == 0) ptx::mbar_arrive_at(&bars[kFull + st], leader, rank);
+                __syncwarp();
+            }
+            for (int jj = max(0, nchunks - kStages); jj < nchunks; ++jj)
+                if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
+                    break;
         } else if (warp == kWarpMma) {
-            // ---------------- MMA issuer (whole warp loops; lane 0 issues) ----------------
+            // ---------------- even CTA: the pair's MMA issuer ----------------
             // tcgen05.mma instructions from one thread execute in issue order, so Q K^T of
             // chunk j + 2 (issued after P V of chunk j) cannot overwrite P_j before it is read.
-            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(kRows, kChunk, false, false);
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, kHeadDim, false, true);
+            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(2 * kRows, kChunk, false, false);
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(2 * kRows, kHeadDim, false, true);
             bool ok = ptx::mbar_wait_warp(&bars[kQReady], 0, abort_flag, S.status);
             ptx::tc_fence_after();
             for (int j = 0; ok && j <= nchunks; ++j) {
                 if (j < nchunks) {
                     const int st = j % kStages;
-                    if (!ptx::mbar_wait_warp(&bars[kKFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
+                    if (!ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
+                    clear_stale_v(j, st);
                     ptx::tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t k_base = ptx::smem_u32(smem + kSmemK + st * kKVBytes);
+                        const uint32_t k_base = ptx::smem_u32(smem + st * kStageBytes);
                         const uint32_t d = tmem + ((j & 1) ? kColS1 : kColS0);
                         for (int ks = 0; ks < kHeadDim / 16; ++ks) {
                             // 16 dims = 32 bytes inside the 128-byte swizzle atom of slab ks / 4
-                            const uint64_t bd = ptx::smem_desc(k_base + (ks >> 2) * kSlabKV + (ks & 3) * 32, 16,
-                                                               1024, ptx::kSwizzle128B);
-                            ptx::mma_ts(d, tmem + kColQ + 8 * ks, bd, idesc_qk, ks > 0 ? 1u : 0u);
+                            const uint64_t bd = ptx::smem_desc(k_base + (ks >> 2) * kSlabK + (ks & 3) * 32, 16, 1024,
+                                                               ptx::kSwizzle128B);
+                            ptx::mma_ts2(d, tmem + kColQ + 8 * ks, bd, idesc_qk, ks > 0 ? 1u : 0u);
                         }
-                        ptx::mma_commit(&bars[kSFull + (j & 1)]);
+                        ptx::mma_commit2_mc(&bars[kSFull + (j & 1)], pair_mask);
                     }
                     __syncwarp();
                 }
                 if (j >= 1) {
                     const int jj = j - 1, st = jj % kStages;
                     if (!ptx::mbar_wait_warp(&bars[kPFull + (jj & 1)], (jj >> 1) & 1, abort_flag, S.status)) break;
-                    if (!ptx::mbar_wait_warp(&bars[kVFull + st], (jj / kStages) & 1, abort_flag, S.status)) break;
-                    // rows past the valid keys may hold stale bytes: zero them so P = 0 times V stays 0
-                    int nvalid;
-                    if (jj < n_ring) nvalid = fill - kChunk * jj;
-                    else if (jj < n_ring + n_blk) nvalid = n - kChunk * (jj - n_ring);
-                    else nvalid = bank_fill - kChunk * (jj - n_ring - n_blk);
-                    if (nvalid < kChunk) {
-                        uint8_t* vst = smem + kSmemV + st * kKVBytes;
-                        const int nz = (kChunk - nvalid) * 8;   // 16-byte pieces per slab
-                        for (int e = lane; e < 4 * nz; e += 32) {
-                            const int slab = e / nz, piece = e % nz;
-                            reinterpret_cast<uint4*>(vst + slab * kSlabKV + nvalid * 128)[piece] =
-                                make_uint4(0, 0, 0, 0);
-                        }
-                        ptx::fence_proxy_async_smem();
-                    }
-                    __syncwarp();
                     ptx::tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t v_base = ptx::smem_u32(smem + kSmemV + st * kKVBytes);
+                        const uint32_t v_base = ptx::smem_u32(smem + st * kStageBytes + kKHalfBytes);
                         const uint32_t a_col = tmem + ((jj & 1) ? kColS1 : kColS0);
                         for (int ks = 0; ks < kChunk / 16; ++ks) {
-                            const uint64_t bd =
-                                ptx::smem_desc(v_base + ks * 16 * 128, kSlabKV, 1024, ptx::kSwizzle128B);
-                            ptx::mma_ts(tmem + kColO, a_col + 8 * ks, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
+                            const uint64_t bd = ptx::smem_desc(v_base + ks * 16 * 128, kSlabV, 1024, ptx::kSwizzle128B);
+                            ptx::mma_ts2(tmem + kColO, a_col + 8 * ks, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
                         }
-                        ptx::mma_commit(&bars[kKVEmpty + st]);
-                        ptx::mma_commit(&bars[kODone]);
+                        ptx::mma_commit2_mc(&bars[kEmpty + st], pair_mask);
+                        ptx::mma_commit2_mc(&bars[kODone], pair_mask);
                     }
                     __syncwarp();
                 }
             }
-            // the producer never waits on the last stages' kv_empty phases: consume them here
-            // so that no commit is still pending when the CTA moves on
+            if (ok && lane == 0) ptx::mma_commit2_mc(&bars[kOFinal], pair_mask);
+            __syncwarp();
+            // consume the last stages' empty phases (the producer never waits on them) so that no
+            // commit is still pending when the CTA moves on
             for (int jj = max(0, nchunks - kStages); ok && jj < nchunks; ++jj)
-                if (!ptx::mbar_wait_warp(&bars[kKVEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
+                if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
                     break;
-        } else {
+        } else if (warp < 8) {
             // ---------------- softmax: thread = (row, half) ----------------
             const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
             {
@@ -278,121 +319,150 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bars[kQReady]);
+                if (lane == 0) ptx::mbar_arrive_at(&bars[kQReady], leader, rank);
+                // this half's part of q . w_g for the gate (the Q row is read again, from L1),
+                // while the first Q K^T runs
+                const float4* wrow = reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + 128 * wg);
+                float gd = 0.f;
+#pragma unroll 2
+                for (int e = 0; e < 16; ++e) {
+                    const uint4 u = __ldg(qrow + e);
+                    const float4 w0 = __ldg(wrow + 2 * e), w1 = __ldg(wrow + 2 * e + 1);
+                    gd += __uint_as_float(u.x << 16) * w0.x + __uint_as_float(u.x & 0xffff0000u) * w0.y +
+                          __uint_as_float(u.y << 16) * w0.z + __uint_as_float(u.y & 0xffff0000u) * w0.w +
+                          __uint_as_float(u.z << 16) * w1.x + __uint_as_float(u.z & 0xffff0000u) * w1.y +
+                          __uint_as_float(u.w << 16) * w1.z + __uint_as_float(u.w & 0xffff0000u) * w1.w;
+                }
+                xch[kXchGate + wg * 128 + row] = gd;
+                ptx::named_bar_sync(1, kSoftmaxThreads);
+                if (wg == 0) {
+                    const float gsum = xch[kXchGate + row] + xch[kXchGate + 128 + row];
+                    xch[kXchGate + row] = tanhf(gsum + a.b_g[head]);
+                }
             }
             const int pq = s + tok;                    // query position
             const int w = (s - 1) % S.R;               // slot of position s - 1 (s >= 1)
             const int base_pos = s - 1 - w;
             const float qs = a.qscale;
-            float m_used = -CUDART_INF_F;
+            // which of keys [32 h, 32 h + 32) of chunk j this row sees, one bit per key
+            auto vis32 = [&](int j, int h) -> uint32_t {
+                if (j < n_ring) {
+                    const int slot0 = kChunk * j + 32 * h;
+                    if (slot0 >= fill) return 0u;
+                    const bool all_valid = slot0 + 31 < fill;
+                    const bool wraps = (slot0 <= w) && (w < slot0 + 31) && (fill == S.R);
+                    const int first = wraps ? w + 1 : slot0;   // the oldest slot of the range
+                    const int pk_min = base_pos + first - (first > w ? S.R : 0);
+                    if (all_valid && pk_min >= pq - S.R) return 0xffffffffu;
+                    uint32_t v = 0;
+#pragma unroll 4
+                    for (int i = 0; i < 32; ++i) {
+                        const int slot = slot0 + i;
+                        const int pk = base_pos + slot - (slot > w ? S.R : 0);
+                        v |= (uint32_t)((slot < fill) && (pk >= pq - S.R)) << i;
+                    }
+                    return v;
+                }
+                if (j < n_ring + n_blk) {
+                    const int t0 = kChunk * (j - n_ring) + 32 * h;
+                    if (t0 > tok || t0 >= n) return 0u;
+                    const int last = min(tok, n - 1) - t0;     // keys t0 .. t0 + last are visible
+                    return last >= 31 ? 0xffffffffu : ((2u << last) - 1u);
+                }
+                const int a0 = kChunk * (j - n_ring - n_blk) + 32 * h;
+                if (a0 >= bank_fill) return 0u;
+                return (bank_fill - a0 >= 32) ? 0xffffffffu : ((1u << (bank_fill - a0)) - 1u);
+            };
+            // The two warpgroups take alternate chunks (this one: j = wg, wg + 2, ...), each a whole
+            // row of 64 keys. The reference max is handed from chunk to chunk through shared memory
+            // (named barrier 2 + wg: this group's value is ready); each group keeps its own row sum
+            // against the reference of its latest chunk.
+            const uint32_t scol = wg ? kColS1 : kColS0;
+            float m_w = -CUDART_INF_F;
             bool ok = true;
-            // Every softmax thread runs every iteration and every named barrier, also after an
-            // abort (then without touching tensor memory), so no thread is left waiting at one.
-            for (int j = 0; j < nchunks; ++j) {
-                const int sb = j & 1;
-                if (ok) ok = ptx::mbar_wait_warp(&bars[kSFull + sb], (j >> 1) & 1, abort_flag, S.status);
+            for (int j = wg; j < nchunks; j += 2) {
+                const uint32_t vlo = vis32(j, 0), vhi = vis32(j, 1);
+                if (ok) ok = ptx::mbar_wait_warp(&bars[kSFull + wg], (j >> 1) & 1, abort_flag, S.status);
                 ok = __all_sync(0xffffffffu, ok);
-                uint32_t sr[32];
+                uint32_t sa[32], sb[32];   // keys [0, 32) and [32, 64)
                 if (ok) {
                     ptx::tc_fence_after();
-                    ptx::tmem_ld32(lane_addr + (sb ? kColS1 : kColS0) + 32 * wg, sr);
+                    ptx::tmem_ld32(lane_addr + scol, sa);
+                    ptx::tmem_ld32(lane_addr + scol + 32, sb);
                     ptx::tmem_wait_ld();
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) sr[i] = 0u;
+                    for (int i = 0; i < 32; ++i) sa[i] = sb[i] = 0u;
                 }
-                // visibility of this thread's 32 keys: 0 all visible, 1 none, 2 per key
-                int mode;
-                uint32_t vis = 0;
-                if (j < n_ring) {
-                    const int slot0 = kChunk * j + 32 * wg;
-                    if (slot0 >= fill) {
-                        mode = 1;
-                    } else {
-                        const bool all_valid = slot0 + 31 < fill;
-                        const bool wraps = (slot0 <= w) && (w < slot0 + 31) && (fill == S.R);
-                        const int first = wraps ? w + 1 : slot0;            // the oldest slot of the range
-                        const int pk_min = base_pos + first - (first > w ? S.R : 0);
-                        mode = (all_valid && pk_min >= pq - S.R) ? 0 : 2;
-                        if (mode == 2) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const int slot = slot0 + i;
-                                const int pk = base_pos + slot - (slot > w ? S.R : 0);
-                                vis |= (uint32_t)((slot < fill) && (pk >= pq - S.R)) << i;
-                            }
-                        }
-                    }
-                } else if (j < n_ring + n_blk) {
-                    const int t0 = kChunk * (j - n_ring) + 32 * wg;
-                    if (t0 > tok || t0 >= n) {
-                        mode = 1;
-                    } else if (t0 + 31 <= tok && t0 + 31 < n) {
-                        mode = 0;
-                    } else {
-                        mode = 2;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) vis |= (uint32_t)((t0 + i <= tok) && (t0 + i < n)) << i;
-                    }
-                } else {
-                    const int a0 = kChunk * (j - n_ring - n_blk) + 32 * wg;
-                    if (a0 >= bank_fill) {
-                        mode = 1;
-                    } else if (a0 + 31 < bank_fill) {
-                        mode = 0;
-                    } else {
-                        mode = 2;
-                        vis = (bank_fill - a0 >= 32) ? 0xffffffffu : ((1u << (bank_fill - a0)) - 1u);
-                    }
-                }
-                if (mode == 0) vis = 0xffffffffu;
-                // the row max over both halves (raw scores; the scale is positive)
+#define SR(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : sb[(i) & 31])
+                const bool full = (vlo & vhi) == 0xffffffffu;
+                // the chunk's row max (raw scores; the scale is positive)
                 float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-                if (mode != 1) {
+                if (full) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float v = ((vis >> i) & 1u) ? __uint_as_float(sr[i]) : -CUDART_INF_F;
-                        m4[i & 3] = fmaxf(m4[i & 3], v);
+                    for (int i = 0; i < 64; ++i) m4[i & 3] = fmaxf(m4[i & 3], SR(i));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const uint32_t bit = ((i < 32 ? vlo : vhi) >> (i & 31)) & 1u;
+                        m4[i & 3] = fmaxf(m4[i & 3], bit ? SR(i) : -CUDART_INF_F);
                     }
                 }
-                float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qs;
-                xch[(sb * 2 + wg) * 128 + row] = mloc;
-                ptx::named_bar_sync(1, kSoftmaxThreads);
-                mloc = fmaxf(mloc, xch[(sb * 2 + (wg ^ 1)) * 128 + row]);
-                float m_new = m_used;
+                const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qs;
+                float m_prev = -CUDART_INF_F;          // the reference O holds after chunk j - 1
+                if (j >= 1) {
+                    ptx::named_bar_sync(2 + (wg ^ 1), kSoftmaxThreads);
+                    m_prev = xch[row];
+                }
+                float m_new = m_prev;
                 bool resc = false;
-                if (mloc > m_used + 8.f) {
-                    resc = (m_used != -CUDART_INF_F);
+                if (mloc > m_prev + 8.f) {
+                    resc = (m_prev != -CUDART_INF_F);
                     m_new = mloc;
                 }
-                const float fac = resc ? fast_ex2(m_used - m_new) : 1.f;
+                if (j + 1 < nchunks) {
+                    xch[row] = m_new;
+                    ptx::named_bar_arrive(2 + wg, kSoftmaxThreads);
+                }
                 const float mref = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-                m_used = m_new;
+                const float fac_l = (m_w == m_new) ? 1.f : (m_w == -CUDART_INF_F ? 0.f : fast_ex2(m_w - m_new));
+                m_w = m_new;
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[16];
-                if (mode == 1) {
+                uint32_t pa[16], pb[16];
+                if (full) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                    for (int i = 0; i < 32; ++i) {
+                        const float e0 = fast_ex2(fmaf(SR(2 * i), qs, -mref));
+                        const float e1 = fast_ex2(fmaf(SR(2 * i + 1), qs, -mref));
+                        s4[i & 3] += e0 + e1;
+                        (i < 16 ? pa[i & 15] : pb[i & 15]) = pack_bf16(e0, e1);
+                    }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float e0 = fast_ex2(fmaf(__uint_as_float(sr[2 * i]), qs, -mref));
-                        float e1 = fast_ex2(fmaf(__uint_as_float(sr[2 * i + 1]), qs, -mref));
-                        e0 = ((vis >> (2 * i)) & 1u) ? e0 : 0.f;
-                        e1 = ((vis >> (2 * i + 1)) & 1u) ? e1 : 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t bits = ((i < 16 ? vlo : vhi) >> ((2 * i) & 31)) & 3u;
+                        float e0 = fast_ex2(fmaf(SR(2 * i), qs, -mref));
+                        float e1 = fast_ex2(fmaf(SR(2 * i + 1), qs, -mref));
+                        e0 = (bits & 1u) ? e0 : 0.f;
+                        e1 = (bits & 2u) ? e1 : 0.f;
                         s4[i & 3] += e0 + e1;
-                        pk[i] = pack_bf16(e0, e1);
+                        (i < 16 ? pa[i & 15] : pb[i & 15]) = pack_bf16(e0, e1);
                     }
                 }
-                l = l * fac + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                if (ok && j >= 1) ok = ptx::mbar_wait_warp(&bars[kODone], (j - 1) & 1, abort_flag, S.status);
+                l = l * fac_l + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                // O may be rescaled only once P V of chunk j - 1 has completed. S of chunk j was
+                // committed after P V of chunk j - 2, so at most that one phase is outstanding.
+                const bool rescale_warp = __any_sync(0xffffffffu, resc);
+                if (ok && rescale_warp)
+                    ok = ptx::mbar_wait_warp(&bars[kODone], (j - 1) & 1, abort_flag, S.status);
                 if (!ok) continue;
                 ptx::tc_fence_after();
-                if (__any_sync(0xffffffffu, resc)) {
+                if (rescale_warp) {
+                    const float fac = resc ? fast_ex2(m_prev - m_new) : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t o[32];
-                        const uint32_t col = kColO + 128 * wg + 32 * c;
+                        const uint32_t col = kColO + 32 * c;
                         ptx::tmem_ld32(lane_addr + col, o);
                         ptx::tmem_wait_ld();
 #pragma unroll
@@ -400,110 +470,118 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::tmem_st32(lane_addr + col, o);
                     }
                 }
-                ptx::tmem_st16(lane_addr + (sb ? kColS1 : kColS0) + 16 * wg, pk);
+#undef SR
+                ptx::tmem_st16(lane_addr + scol, pa);
+                ptx::tmem_st16(lane_addr + scol + 16, pb);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bars[kPFull + sb]);
+                if (lane == 0) ptx::mbar_arrive_at(&bars[kPFull + wg], leader, rank);
             }
-            // both halves of a row used the same reference max: the row sum is the sum of halves
-            xch[(4 + wg) * 128 + row] = l;
+            // the row sum over both groups, on the last chunk's reference (references only grow)
+            xch[kXchEndL + wg * 128 + row] = l;
+            xch[kXchEndM + wg * 128 + row] = m_w;
             ptx::named_bar_sync(1, kSoftmaxThreads);
-            l += xch[(4 + (wg ^ 1)) * 128 + row];
-            if (ok && ptx::mbar_wait_warp(&bars[kODone], (nchunks - 1) & 1, abort_flag, S.status)) {
-                ptx::tc_fence_after();
-                const float inv = (l > 0.f) ? 1.f / l : 0.f;
-                float4* dst = reinterpret_cast<float4*>(own_rows + (size_t)row * kHeadDim + 128 * wg);
+            {
+                const float lo = xch[kXchEndL + (wg ^ 1) * 128 + row];
+                const float mo = xch[kXchEndM + (wg ^ 1) * 128 + row];
+                const float mf = fmaxf(m_w, mo);
+                float lt = 0.f;
+                if (m_w != -CUDART_INF_F) lt += l * fast_ex2(m_w - mf);
+                if (mo != -CUDART_INF_F) lt += lo * fast_ex2(mo - mf);
+                l = lt;
+            }
+            const bool done = ok && ptx::mbar_wait_warp(&bars[kOFinal], 0, abort_flag, S.status);
+            // every MMA of the pair has completed (or the CTA gave up): the K/V stages are free
+            ptx::named_bar_sync(1, kSoftmaxThreads);
+            if (done) ptx::tc_fence_after();
+            const float inv = (done && l > 0.f) ? 1.f / l : 0.f;
+            uint8_t* rrow = smem + (size_t)row * 1024;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                if (done) {
                     ptx::tmem_ld32(lane_addr + kColO + 128 * wg + 32 * c, o);
                     ptx::tmem_wait_ld();
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[c * 8 + i] =
-                            make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                        __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
                 }
-                l = inv;   // from here on: the row's normalisation factor
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int piece = 32 * wg + 8 * c + i;
+                    *reinterpret_cast<float4*>(rrow + ((piece ^ (row & 7)) << 4)) =
+                        make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                    __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+                }
             }
+            ptx::fence_proxy_async_smem();   // the rows leave through a bulk copy
         }
     } else if (warp < 8) {
-        // nothing to read (empty bank): this CTA's rows are zero
-        float4* dst = reinterpret_cast<float4*>(own_rows + (size_t)row * kHeadDim + 128 * wg);
-        for (int c = 0; c < 32; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // nothing to read (empty bank): this CTA's rows are zero (and so is the anchor's gate term)
+        for (int c = 0; c < 32; ++c)
+            *reinterpret_cast<float4*>(smem + (size_t)row * 1024 + ((32 * wg + c) << 4)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (wg == 0) xch[kXchGate + row] = 0.f;
+        ptx::fence_proxy_async_smem();
     }
 
     // ---------------- tail ----------------
-    __threadfence();
+    // The local CTA of this tile combines rows [0, 64), the anchor CTA rows [64, 128): each first
+    // pushes the 64 rows the other one needs into that CTA's free stage area [128 KiB, 192 KiB).
     ptx::tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned old = atomicAdd(S.tickets + bg, (1u << (2 * T)) + (1u << 16));
-        tail_flags[0] = ((old >> (2 * T)) & 3u) != 0u;
-        tail_flags[1] = (int)(old >> 16) == 2 * ntiles - 1;
-    }
-    __syncthreads();
-    const bool partner_done = tail_flags[0] != 0, last_all = tail_flags[1] != 0;
-    if (partner_done && warp < 8) {
-        // out = local + gate * anchor; this thread: one row, one half of the dims
-        __threadfence();
+    ptx::cluster_sync();   // all four CTAs have their rows in shared memory; all tensor memory reads done
+    if (has_work && warp == kWarpMma) {
         ptx::tc_fence_after();
-        const size_t qoff = ((size_t)(b * n + tok) * HQ + head) * kHeadDim;
-        const uint4* qrow = reinterpret_cast<const uint4*>(a.q + qoff) + 16 * wg;
-        const float4* wrow = reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + 128 * wg);
-        float d = 0.f;
-#pragma unroll 4
-        for (int e = 0; e < 16; ++e) {
-            const uint4 qv = __ldg(qrow + e);
-            const float4 w0 = __ldg(wrow + 2 * e), w1 = __ldg(wrow + 2 * e + 1);
-            d += __uint_as_float(qv.x << 16) * w0.x + __uint_as_float(qv.x & 0xffff0000u) * w0.y +
-                 __uint_as_float(qv.y << 16) * w0.z + __uint_as_float(qv.y & 0xffff0000u) * w0.w +
-                 __uint_as_float(qv.z << 16) * w1.x + __uint_as_float(qv.z & 0xffff0000u) * w1.y +
-                 __uint_as_float(qv.w << 16) * w1.z + __uint_as_float(qv.w & 0xffff0000u) * w1.w;
-        }
-        xch[(6 + wg) * 128 + row] = d;
-        ptx::named_bar_sync(1, kSoftmaxThreads);
-        d += xch[(6 + (wg ^ 1)) * 128 + row];
-        const float gate = tanhf(d + a.b_g[head]);
-        // own result scaled by its normalisation (0 when there was nothing to read)
-        const float c_own = (phase == 0 ? 1.f : gate) * (has_work ? l : 0.f);
-        const float c_par = phase == 0 ? gate : 1.f;
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        const float4* prow = reinterpret_cast<const float4*>(partner_rows + (size_t)row * kHeadDim + 128 * wg);
-        uint4* orow = reinterpret_cast<uint4*>(a.out + qoff) + 16 * wg;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            if (has_work) {
-                ptx::tmem_ld32(lane_addr + kColO + 128 * wg + 32 * c, o);
-                ptx::tmem_wait_ld();
-            } else {
+        ptx::tmem_dealloc2(tmem, kTmemCols);
+    }
+    const uint32_t peer = rank ^ 2u;
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(&bars[kXfer], 64 * 1024);
+        const uint32_t src = ptx::smem_u32(smem) + (uint32_t)(64 * (1 - phase)) * 1024u;
+        const uint32_t dst = ptx::cluster_map(ptx::smem_u32(smem) + 128u * 1024u, peer);
+        const uint32_t rbar = ptx::cluster_map(ptx::smem_u32(&bars[kXfer]), peer);
+        ptx::bulk_copy_to_peer(dst, src, 64 * 1024, rbar);
+        ptx::bulk_commit();
+    }
+    if (warp < 8) {
+        // 4 threads per row, 64 dims each
+        const int crow = 64 * phase + (tid >> 2), qd = tid & 3;
+        const int ctok = kTileTok * T + (crow >> 2), chead = g * kQPerGroup + (crow & 3);
+        const size_t qoff = ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim + 64 * qd;
+        const float gate = xch[kXchGate + crow];
+        const bool got = ptx::mbar_wait_warp(&bars[kXfer], 0, abort_flag, S.status);
+        const uint8_t* prow = smem + 128 * 1024 + (size_t)(crow - 64 * phase) * 1024;
+        const uint8_t* mrow = smem + (size_t)crow * 1024;
+        uint4* orow = reinterpret_cast<uint4*>(a.out + qoff);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) o[i] = 0u;
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t off0 = (uint32_t)(((16 * qd + 2 * e) ^ (crow & 7)) << 4);
+            const uint32_t off1 = (uint32_t)(((16 * qd + 2 * e + 1) ^ (crow & 7)) << 4);
+            const float4 m0 = *reinterpret_cast<const float4*>(mrow + off0);
+            const float4 m1 = *reinterpret_cast<const float4*>(mrow + off1);
+            float4 t0 = make_float4(0.f, 0.f, 0.f, 0.f), t1 = t0;
+            if (got) {
+                t0 = *reinterpret_cast<const float4*>(prow + off0);
+                t1 = *reinterpret_cast<const float4*>(prow + off1);
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 p0 = __ldcg(prow + 8 * c + 2 * e), p1 = __ldcg(prow + 8 * c + 2 * e + 1);
-                const float* ov = reinterpret_cast<const float*>(o) + 8 * e;
-                uint4 r;
-                r.x = pack_bf16(c_own * ov[0] + c_par * p0.x, c_own * ov[1] + c_par * p0.y);
-                r.y = pack_bf16(c_own * ov[2] + c_par * p0.z, c_own * ov[3] + c_par * p0.w);
-                r.z = pack_bf16(c_own * ov[4] + c_par * p1.x, c_own * ov[5] + c_par * p1.y);
-                r.w = pack_bf16(c_own * ov[6] + c_par * p1.z, c_own * ov[7] + c_par * p1.w);
-                orow[4 * c + e] = r;
-            }
+            const float4 l0 = phase == 0 ? m0 : t0, l1 = phase == 0 ? m1 : t1;
+            const float4 c0 = phase == 0 ? t0 : m0, c1 = phase == 0 ? t1 : m1;
+            uint4 r;
+            r.x = pack_bf16(l0.x + gate * c0.x, l0.y + gate * c0.y);
+            r.y = pack_bf16(l0.z + gate * c0.z, l0.w + gate * c0.w);
+            r.z = pack_bf16(l1.x + gate * c1.x, l1.y + gate * c1.y);
+            r.w = pack_bf16(l1.z + gate * c1.z, l1.w + gate * c1.w);
+            orow[e] = r;
         }
     }
-    if (has_work) {
-        ptx::tc_fence_before();
-        __syncthreads();
-        if (warp == kWarpMma) {
-            ptx::tc_fence_after();
-            ptx::tmem_dealloc(tmem, kTmemCols);
-        }
+    if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
+    __threadfence();
+    if (tid == 0) {
+        const unsigned old = atomicAdd(S.tickets + bg, 1u);
+        *tail_flag = (int)old == 2 * ntiles - 1;
     }
-    if (!last_all) return;
+    __syncthreads();
+    if (*tail_flag == 0) return;
 
     // ---------------- last CTA of (b, g): commit the block, then the forced admit ----------------
     __threadfence();
@@ -575,22 +653,25 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d1, uint64_t d2, uint64
 }  // namespace
 
 size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok) {
-    const size_t ntiles = (size_t)(n_tok + kTileTok - 1) / kTileTok;
-    return (size_t)cfg.batch * cfg.n_groups * ntiles * 2 * kRows * kHeadDim * sizeof(float);
+    // the tile CTAs exchange their rows through distributed shared memory: no device scratch
+    (void)cfg;
+    (void)n_tok;
+    return 256;
 }
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const LayerView& s = a.s;
     const int B = s.B, G = s.G, n = a.n_tok;
-    if (n % kTileTok != 0 || n > kMaxTiles * kTileTok || n > s.R) return cudaErrorNotSupported;
+    // tiles come in pairs (64 tokens); the ticket counts 2 * ntiles arrivals
+    if (n % (kTilesPerCluster * kTileTok) != 0 || n > 256 || n > s.R) return cudaErrorNotSupported;
     const int ntiles = n / kTileTok;
     Tmaps tm;
     const uint64_t row = (uint64_t)kHeadDim * 2;
-    bool ok = make_map(&tm.k, a.k, G, (uint64_t)B * n, row, row * G, 1, kChunk) &&
+    bool ok = make_map(&tm.k, a.k, G, (uint64_t)B * n, row, row * G, 1, kHalfKeys) &&
               make_map(&tm.v, a.v, G, (uint64_t)B * n, row, row * G, 1, kChunk) &&
-              make_map(&tm.ring_k, s.ring_k, s.R, (uint64_t)B * G, row, row * s.R, kChunk, 1) &&
+              make_map(&tm.ring_k, s.ring_k, s.R, (uint64_t)B * G, row, row * s.R, kHalfKeys, 1) &&
               make_map(&tm.ring_v, s.ring_v, s.R, (uint64_t)B * G, row, row * s.R, kChunk, 1) &&
-              make_map(&tm.bank_k, s.bank_k, s.A, (uint64_t)B * G, row, row * s.A, kChunk, 1) &&
+              make_map(&tm.bank_k, s.bank_k, s.A, (uint64_t)B * G, row, row * s.A, kHalfKeys, 1) &&
               make_map(&tm.bank_v, s.bank_v, s.A, (uint64_t)B * G, row, row * s.A, kChunk, 1);
     if (!ok) return cudaErrorInvalidValue;
     static bool configured = false;
@@ -599,6 +680,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured = true;
     }
+    // grid x: clusters of 4 CTAs, one per pair of tiles; ranks (local, local, anchor, anchor)
     prefill_kernel<<<dim3(2 * ntiles, G, B), kThreads, kSmemBytes, stream>>>(tm, a, ntiles);
     return cudaGetLastError();
 }

@@ -229,7 +229,7 @@ RMA_API int rma_admit(rma_state* st, int layer, int force, void* stream);
  *   out         bf16 [batch][n_tok][n_groups*q_per_group][head_dim]  (written)
  *   ws          workspace of rma_workspace_bytes(st, n_tok) bytes
  * One launch: the admit runs inside it once every read of the block is done.
- * This build requires n_tok == pend_slots, n_tok a multiple of 32, at most
+ * This build requires n_tok == pend_slots, n_tok a multiple of 64, at most
  * 256 and at most ring_slots (RMA_ERR_UNSUPPORTED otherwise).  Alignment as
  * in rma_decode_step. */
 RMA_API int rma_prefill_block(rma_state* st, int layer, int n_tok,

@@ -160,3 +160,19 @@ def workload_counters(kind: str, n_layers: int, batch: int, n_groups: int, ring_
         raise ValueError(kind)
     return {"pos": np.array(pos, dtype=np.int64), "bank_fill": np.array(bank, dtype=np.int64),
             "pend_fill": np.array(pend, dtype=np.int64)}
+
+
+def aligned_ramp(lead_shape, n_rows: int, head_dim: int, seed: int, lo: float, hi: float,
+                 noise: float = 0.25, device="cpu") -> torch.Tensor:
+    """BF16 rows along one shared direction with magnitudes growing linearly from lo to hi.
+
+    Row i of [*lead_shape, n_rows, head_dim] is ``c_i u + noise z`` with u ~ N(0, 1)^D drawn from
+    ``seed`` (the same u for every call with that seed), c_i = lo + (hi - lo) i / (n_rows - 1) and
+    z ~ N(0, 1).  Queries drawn with lo = hi = 1 and keys with a wide ramp give scores that keep
+    rising along the rows, so a running maximum moves many times.
+    """
+    u = torch.randn((head_dim,), generator=_gen(seed, "cpu"), dtype=torch.float32).to(device)
+    c = torch.linspace(float(lo), float(hi), n_rows, dtype=torch.float32, device=device)
+    z = torch.randn(tuple(lead_shape) + (n_rows, head_dim), generator=_gen(int(seed) + 1, device),
+                    device=device, dtype=torch.float32)
+    return (c[:, None] * u + noise * z).to(torch.bfloat16)

@@ -122,3 +122,37 @@ def test_prefill_then_decode_handoff():
         oracle.admit(ost, 0)
         assert output_error(to_np(out), r) <= TOL
     assert_state_equal(gpu_state_np(st), ost, "after handoff")
+
+
+def test_prefill_rescales_when_scores_keep_rising():
+    """Keys along the queries' direction with growing magnitude: the running max of every row moves
+    many times (ring slots, then the block, then a rising bank), so O and the row sums are rescaled
+    repeatedly, in both query groups."""
+    rma = lib()
+    cfg = oracle.Config(batch=2, n_layers=1)
+    st, ost = make_pair(cfg, seed=31, pos=3000, bank_fill=1024, pend_fill=0)
+    L, B, G, D = 1, cfg.batch, cfg.n_groups, cfg.head_dim
+    ring_k = si.aligned_ramp((L, B, G), cfg.ring_slots, D, seed=310, lo=0.0, hi=1.5)
+    bank_k = si.aligned_ramp((L, B, G), cfg.bank_slots, D, seed=310, lo=-0.5, hi=2.0)
+    for name, t in (("ring_k", ring_k), ("bank_k", bank_k)):
+        getattr(st, name).copy_(t)
+        getattr(ost, name)[...] = to_np(t)
+    n = cfg.pend_slots
+    x = si.prefill_inputs(B, n, G, cfg.q_per_group, D, seed=311)
+    x["q"] = si.aligned_ramp((B,), n * G * cfg.q_per_group, D, seed=310, lo=1.0, hi=1.0).reshape(
+        B, n, G * cfg.q_per_group, D)
+    x["k"] = si.aligned_ramp((B, G), n, D, seed=310, lo=1.5, hi=2.5).permute(0, 2, 1, 3).contiguous()
+    w, b = si.gate_params(1, 16, 256, seed=31)
+    w, b = w[0].cuda(), si.f32_normal((16,), 32, std=0.5).cuda()
+    xd = {k: v.cuda() for k, v in x.items()}
+    out = torch.empty(B, n, G * cfg.q_per_group, D, dtype=torch.bfloat16, device="cuda")
+    rma.prefill_block(st, 0, xd["q"], xd["k"], xd["v"], xd["cand_k"], xd["cand_v"], xd["cand_score"], w, b, out,
+                      st.workspace(n))
+    xn = {k: to_np(v) for k, v in x.items()}
+    ref = oracle.prefill_block(ost, 0, xn["q"], xn["k"], xn["v"], xn["cand_k"], xn["cand_v"], xn["cand_score"],
+                               to_np(w), to_np(b))
+    torch.cuda.synchronize()
+    err = output_error(to_np(out), ref)
+    assert err <= TOL, f"output error {err}"
+    assert_state_equal(gpu_state_np(st), ost, "rising scores")
+    assert rma.get_status(st) == 0
