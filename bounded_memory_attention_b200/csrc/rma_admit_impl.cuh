@@ -43,6 +43,31 @@ __host__ __device__ constexpr size_t admit_scratch_bytes(int A, int P) {
     return ((size_t)(A + P) * 8 + (size_t)(A + P) + 15) / 16 * 16 + (size_t)(2 * P + 256 + 64) * 4;
 }
 
+// Copy `total` 16-byte pieces with the whole CTA (NT threads): piece e goes from src(e) to
+// dst(e), given by where(e, src, dst).  Each thread issues U loads before the first of its
+// stores so that U pieces per thread are in flight at once.  The loads go through L2 only
+// (.cg): the source may have been written earlier in the same launch by another CTA.
+template <int NT, int U, class Where>
+__device__ __forceinline__ void copy_pieces(int total, Where where) {
+    for (int e0 = threadIdx.x; e0 < total; e0 += NT * U) {
+        uint4 v[U];
+        uint4* d[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = e0 + u * NT;
+            d[u] = nullptr;
+            if (e < total) {
+                const uint4* src;
+                where(e, src, d[u]);
+                v[u] = __ldcg(src);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (d[u]) *d[u] = v[u];
+    }
+}
+
 // Exclusive prefix sum of one int per thread over NT threads; *total gets the sum.
 template <int NT>
 __device__ __forceinline__ int admit_block_scan(int v, int* warp_tot, int* total) {
@@ -218,13 +243,18 @@ __device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t*
     uint4* bk = reinterpret_cast<uint4*>(s.bank_k + (size_t)bg * A * kHeadDim);
     uint4* bv = reinterpret_cast<uint4*>(s.bank_v + (size_t)bg * A * kHeadDim);
     constexpr int kChunks = kRowBytes / 16;   // 32 per row
-    for (int e = tid; e < n_adm * 2 * kChunks; e += NT) {
+    copy_pieces<NT, 8>(n_adm * 2 * kChunks, [&](int e, const uint4*& from_p, uint4*& to_p) {
         const int j = e / (2 * kChunks);
         const int c = e % (2 * kChunks);
         const int from = src[j], to = dest[j];
-        if (c < kChunks) bk[(size_t)to * kChunks + c] = pk[(size_t)from * kChunks + c];
-        else bv[(size_t)to * kChunks + (c - kChunks)] = pv[(size_t)from * kChunks + (c - kChunks)];
-    }
+        if (c < kChunks) {
+            from_p = pk + (size_t)from * kChunks + c;
+            to_p = bk + (size_t)to * kChunks + c;
+        } else {
+            from_p = pv + (size_t)from * kChunks + (c - kChunks);
+            to_p = bv + (size_t)to * kChunks + (c - kChunks);
+        }
+    });
     for (int j = tid; j < n_adm; j += NT) s.bank_score[(size_t)bg * A + dest[j]] = pscore[src[j]];
     if (tid == 0) {
         int32_t* cnt = s.counters + bg * 4;

@@ -65,17 +65,23 @@ constexpr int kSlabV = kChunk * 128;                  // 64 keys x 64 dims = 8 K
 constexpr int kKHalfBytes = 4 * kSlabK;               // 16 KiB: this CTA's keys, all 256 dims
 constexpr int kVHalfBytes = 2 * kSlabV;               // 16 KiB: all 64 keys, this CTA's 128 dims
 constexpr int kStageBytes = kKHalfBytes + kVHalfBytes;
-constexpr int kStages = 6;
-constexpr int kSmemBar = kStages * kStageBytes;       // 192 KiB
+constexpr int kStages = 5;
+constexpr int kSmemP = kStages * kStageBytes;         // 160 KiB: P of the two softmax groups
+constexpr int kPBytes = 128 * 128;                    // 128 rows x 64 keys (BF16), 128-byte swizzle
+constexpr int kSmemBar = kSmemP + 2 * kPBytes;        // 192 KiB
 // softmax exchange (floats): the reference max handed between the groups [128] at 0, each
 // group's final reference max [2][128] at 128 and row sum [2][128] at 512, the gate [128] at 768
 // (first the two halves' partial dot products [2][128], then the gate itself in the first)
 constexpr int kSmemXch = kSmemBar + 512;
-constexpr int kSmemBytes = kSmemXch + 4096 + 1024;    // + 1 KiB for alignment
+constexpr int kSmemW = kSmemXch + 4096;               // w_g rows of the group's 4 heads (FP32)
+constexpr int kSmemBytes = kSmemW + 4096 + 1024;      // + 1 KiB for alignment
 constexpr int kXchEndM = 128, kXchEndL = 512, kXchGate = 768;
 constexpr int kSoftmaxThreads = 256;                  // warps 0-7
-constexpr int kWarpTma = 8, kWarpMma = 9;
-constexpr int kThreads = 320;
+// warp 8: TMA producer; warp 9: Q K^T issuer (even CTA) or stale-row cleaner (odd CTA);
+// warp 10: P V issuer (even CTA).  Two issuing warps keep the tensor pipe fed while either
+// one waits on a barrier.
+constexpr int kWarpTma = 8, kWarpQK = 9, kWarpPV = 10;
+constexpr int kThreads = 352;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
 constexpr int kTilesPerCluster = 2;
@@ -89,14 +95,15 @@ struct Tmaps {
 
 enum Bar {
     kQReady = 0,                // even CTA: 16 arrivals (8 warps x 2 CTAs)
-    kFull = 1,                  // [6] even CTA: own loads (tx) + the odd CTA's signal; odd CTA: own loads
-    kEmpty = 7,                 // [6] both: the MMA commit after P V of the chunk in that stage
-    kSFull = 13,                // [2] both: MMA commit after Q K^T
-    kPFull = 15,                // [2] even CTA, one per softmax group: 8 arrivals (4 warps x 2 CTAs)
-    kODone = 17,                // both: MMA commit after P V
-    kXfer = 18,                 // both: the other CTA's half-result rows have landed (tx bytes)
-    kOFinal = 19,               // both: MMA commit after the last P V (one phase)
-    kNumBars = 20
+    kFull = 1,                  // [5] even CTA: own loads (tx) + the odd CTA's signal; odd CTA: own loads
+    kEmpty = 6,                 // [5] both: the MMA commit after P V of the chunk in that stage (the stage,
+                                //     that P buffer and O are free to reuse)
+    kSFull = 11,                // [2] both, one per softmax group: MMA commit after Q K^T
+    kPFull = 13,                // [2] even CTA, per group: P is in shared memory, 8 arrivals (4 warps x 2 CTAs)
+    kSFree = 15,                // [2] even CTA, per group: S has been read, 8 arrivals
+    kXfer = 17,                 // both: the other CTA's half-result rows have landed (tx bytes)
+    kOFinal = 18,               // both: MMA commit after the last P V (one phase)
+    kNumBars = 19
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -165,14 +172,17 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars[kSFull + i], 1);
             ptx::mbar_init(&bars[kPFull + i], 8);
+            ptx::mbar_init(&bars[kSFree + i], 8);
         }
-        ptx::mbar_init(&bars[kODone], 1);
         ptx::mbar_init(&bars[kXfer], 1);
         ptx::mbar_init(&bars[kOFinal], 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (has_work && warp == kWarpMma) {
+    if (tid < kSoftmaxThreads)   // the gate weights of the group's heads, one float4 per thread
+        reinterpret_cast<float4*>(smem + kSmemW)[tid] =
+            __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)g * kQPerGroup * kHeadDim) + tid);
+    if (has_work && warp == kWarpQK) {
         ptx::tmem_alloc2(tmem_holder, kTmemCols);
         ptx::tmem_relinquish2();
     }
@@ -237,7 +247,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-        } else if (warp == kWarpMma && pr == 1) {
+        } else if (warp == kWarpQK && pr == 1) {
             // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
             for (int j = 0; j < nchunks; ++j) {
                 const int st = j % kStages;
@@ -249,49 +259,58 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             for (int jj = max(0, nchunks - kStages); jj < nchunks; ++jj)
                 if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
                     break;
-        } else if (warp == kWarpMma) {
-            // ---------------- even CTA: the pair's MMA issuer ----------------
-            // tcgen05.mma instructions from one thread execute in issue order, so Q K^T of
-            // chunk j + 2 (issued after P V of chunk j) cannot overwrite P_j before it is read.
+        } else if (warp == kWarpQK) {
+            // ---------------- even CTA: Q K^T issuer ----------------
+            // S of chunk j lives in columns kColS0 / kColS1 by j & 1 and P in shared memory, so
+            // Q K^T of chunk j + 2 may start as soon as the softmax group has read S of chunk j.
             constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(2 * kRows, kChunk, false, false);
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(2 * kRows, kHeadDim, false, true);
             bool ok = ptx::mbar_wait_warp(&bars[kQReady], 0, abort_flag, S.status);
             ptx::tc_fence_after();
-            for (int j = 0; ok && j <= nchunks; ++j) {
-                if (j < nchunks) {
-                    const int st = j % kStages;
-                    if (!ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
-                    clear_stale_v(j, st);
-                    ptx::tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t k_base = ptx::smem_u32(smem + st * kStageBytes);
-                        const uint32_t d = tmem + ((j & 1) ? kColS1 : kColS0);
-                        for (int ks = 0; ks < kHeadDim / 16; ++ks) {
-                            // 16 dims = 32 bytes inside the 128-byte swizzle atom of slab ks / 4
-                            const uint64_t bd = ptx::smem_desc(k_base + (ks >> 2) * kSlabK + (ks & 3) * 32, 16, 1024,
-                                                               ptx::kSwizzle128B);
-                            ptx::mma_ts2(d, tmem + kColQ + 8 * ks, bd, idesc_qk, ks > 0 ? 1u : 0u);
-                        }
-                        ptx::mma_commit2_mc(&bars[kSFull + (j & 1)], pair_mask);
-                    }
-                    __syncwarp();
+            for (int j = 0; ok && j < nchunks; ++j) {
+                if (j >= 2) {
+                    ok = ptx::mbar_wait_warp(&bars[kSFree + (j & 1)], ((j - 2) >> 1) & 1, abort_flag, S.status);
+                    if (!ok) break;
                 }
-                if (j >= 1) {
-                    const int jj = j - 1, st = jj % kStages;
-                    if (!ptx::mbar_wait_warp(&bars[kPFull + (jj & 1)], (jj >> 1) & 1, abort_flag, S.status)) break;
-                    ptx::tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t v_base = ptx::smem_u32(smem + st * kStageBytes + kKHalfBytes);
-                        const uint32_t a_col = tmem + ((jj & 1) ? kColS1 : kColS0);
-                        for (int ks = 0; ks < kChunk / 16; ++ks) {
-                            const uint64_t bd = ptx::smem_desc(v_base + ks * 16 * 128, kSlabV, 1024, ptx::kSwizzle128B);
-                            ptx::mma_ts2(tmem + kColO, a_col + 8 * ks, bd, idesc_pv, (jj > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        ptx::mma_commit2_mc(&bars[kEmpty + st], pair_mask);
-                        ptx::mma_commit2_mc(&bars[kODone], pair_mask);
+                const int st = j % kStages;
+                ok = ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status);
+                if (!ok) break;
+                clear_stale_v(j, st);
+                ptx::tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t k_base = ptx::smem_u32(smem + st * kStageBytes);
+                    const uint32_t d = tmem + ((j & 1) ? kColS1 : kColS0);
+                    for (int ks = 0; ks < kHeadDim / 16; ++ks) {
+                        // 16 dims = 32 bytes inside the 128-byte swizzle atom of slab ks / 4
+                        const uint64_t bd = ptx::smem_desc(k_base + (ks >> 2) * kSlabK + (ks & 3) * 32, 16, 1024,
+                                                           ptx::kSwizzle128B);
+                        ptx::mma_ts2(d, tmem + kColQ + 8 * ks, bd, idesc_qk, ks > 0 ? 1u : 0u);
                     }
-                    __syncwarp();
+                    ptx::mma_commit2_mc(&bars[kSFull + (j & 1)], pair_mask);
                 }
+                __syncwarp();
+            }
+        } else if (warp == kWarpPV && pr == 0) {
+            // ---------------- even CTA: P V issuer ----------------
+            // P V of chunk j needs P (which the softmax writes only after reading S of chunk j,
+            // so Q K^T of chunk j has completed) and V (landed before Q K^T of chunk j was issued).
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(2 * kRows, kHeadDim, false, true);
+            bool ok = true;
+            for (int j = 0; ok && j < nchunks; ++j) {
+                const int st = j % kStages;
+                ok = ptx::mbar_wait_warp(&bars[kPFull + (j & 1)], (j >> 1) & 1, abort_flag, S.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t v_base = ptx::smem_u32(smem + st * kStageBytes + kKHalfBytes);
+                    const uint32_t p_base = ptx::smem_u32(smem + kSmemP + (j & 1) * kPBytes);
+                    for (int ks = 0; ks < kChunk / 16; ++ks) {
+                        const uint64_t ad = ptx::smem_desc(p_base + ks * 32, 16, 1024, ptx::kSwizzle128B);
+                        const uint64_t bd = ptx::smem_desc(v_base + ks * 16 * 128, kSlabV, 1024, ptx::kSwizzle128B);
+                        ptx::mma_ss2(tmem + kColO, ad, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    ptx::mma_commit2_mc(&bars[kEmpty + st], pair_mask);
+                }
+                __syncwarp();
             }
             if (ok && lane == 0) ptx::mma_commit2_mc(&bars[kOFinal], pair_mask);
             __syncwarp();
@@ -322,12 +341,12 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 if (lane == 0) ptx::mbar_arrive_at(&bars[kQReady], leader, rank);
                 // this half's part of q . w_g for the gate (the Q row is read again, from L1),
                 // while the first Q K^T runs
-                const float4* wrow = reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + 128 * wg);
+                const float4* wrow = reinterpret_cast<const float4*>(smem + kSmemW) + ((row & 3) * kHeadDim + 128 * wg) / 4;
                 float gd = 0.f;
 #pragma unroll 2
                 for (int e = 0; e < 16; ++e) {
                     const uint4 u = __ldg(qrow + e);
-                    const float4 w0 = __ldg(wrow + 2 * e), w1 = __ldg(wrow + 2 * e + 1);
+                    const float4 w0 = wrow[2 * e], w1 = wrow[2 * e + 1];
                     gd += __uint_as_float(u.x << 16) * w0.x + __uint_as_float(u.x & 0xffff0000u) * w0.y +
                           __uint_as_float(u.y << 16) * w0.z + __uint_as_float(u.y & 0xffff0000u) * w0.w +
                           __uint_as_float(u.z << 16) * w1.x + __uint_as_float(u.z & 0xffff0000u) * w1.y +
@@ -390,6 +409,9 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                     ptx::tmem_ld32(lane_addr + scol, sa);
                     ptx::tmem_ld32(lane_addr + scol + 32, sb);
                     ptx::tmem_wait_ld();
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive_at(&bars[kSFree + wg], leader, rank);   // S may be overwritten
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sa[i] = sb[i] = 0u;
@@ -450,14 +472,20 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
                 l = l * fac_l + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                // O may be rescaled only once P V of chunk j - 1 has completed. S of chunk j was
-                // committed after P V of chunk j - 2, so at most that one phase is outstanding.
+                // O may be rescaled only once P V of chunk j - 1 (the other group's) has completed,
+                // and this group's P buffer is free once P V of chunk j - 2 has; both are the
+                // stage barriers of those chunks.  P V runs in chunk order and this group saw
+                // P V of chunk j - 4 complete, so each barrier is at most one phase behind.
                 const bool rescale_warp = __any_sync(0xffffffffu, resc);
                 if (ok && rescale_warp)
-                    ok = ptx::mbar_wait_warp(&bars[kODone], (j - 1) & 1, abort_flag, S.status);
+                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (j - 1) % kStages], ((j - 1) / kStages) & 1, abort_flag,
+                                             S.status);
+                if (ok && j >= 2)
+                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (j - 2) % kStages], ((j - 2) / kStages) & 1, abort_flag,
+                                             S.status);
                 if (!ok) continue;
-                ptx::tc_fence_after();
                 if (rescale_warp) {
+                    ptx::tc_fence_after();
                     const float fac = resc ? fast_ex2(m_prev - m_new) : 1.f;
 #pragma unroll 1
                     for (int c = 0; c < 8; ++c) {
@@ -469,11 +497,19 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac);
                         ptx::tmem_st32(lane_addr + col, o);
                     }
+                    ptx::tmem_wait_st();
                 }
 #undef SR
-                ptx::tmem_st16(lane_addr + scol, pa);
-                ptx::tmem_st16(lane_addr + scol + 16, pb);
-                ptx::tmem_wait_st();
+                // P row: 64 keys as BF16 = 128 bytes, 16-byte pieces swizzled by the row within its 8-row atom
+                uint8_t* prow = smem + kSmemP + wg * kPBytes + row * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+                        make_uint4(pa[4 * c], pa[4 * c + 1], pa[4 * c + 2], pa[4 * c + 3]);
+                    *reinterpret_cast<uint4*>(prow + (((c + 4) ^ (row & 7)) << 4)) =
+                        make_uint4(pb[4 * c], pb[4 * c + 1], pb[4 * c + 2], pb[4 * c + 3]);
+                }
+                ptx::fence_proxy_async_smem();   // P is read by the tensor cores
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive_at(&bars[kPFull + wg], leader, rank);
@@ -530,7 +566,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     // pushes the 64 rows the other one needs into that CTA's free stage area [128 KiB, 192 KiB).
     ptx::tc_fence_before();
     ptx::cluster_sync();   // all four CTAs have their rows in shared memory; all tensor memory reads done
-    if (has_work && warp == kWarpMma) {
+    if (has_work && warp == kWarpQK) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc2(tmem, kTmemCols);
     }
@@ -575,7 +611,32 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         }
     }
     if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
+
+    // This CTA's share of the candidates goes to pending now (nothing in this launch reads those
+    // slots before the last CTA's admit); the ring write has to wait until every CTA of the group
+    // has read the ring.
+    const bool fits = pend_fill + n <= S.P;
+    constexpr int kPieces = kRowBytes / 16;   // 32 per row
+    const int nct = gridDim.x, share = (n + nct - 1) / nct;
+    const int i0 = min(n, (int)blockIdx.x * share), i1 = min(n, i0 + share);
+    if (fits) {
+        copy_pieces<kThreads, 4>((i1 - i0) * 2 * kPieces, [&](int e, const uint4*& from_p, uint4*& to_p) {
+            const int i = i0 + e / (2 * kPieces), c = e % (2 * kPieces);
+            const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
+            const size_t pd = ((size_t)bg * S.P + pend_fill + i) * kHeadDim;
+            if (c < kPieces) {
+                from_p = reinterpret_cast<const uint4*>(a.cand_k + src) + c;
+                to_p = reinterpret_cast<uint4*>(S.pend_k + pd) + c;
+            } else {
+                from_p = reinterpret_cast<const uint4*>(a.cand_v + src) + (c - kPieces);
+                to_p = reinterpret_cast<uint4*>(S.pend_v + pd) + (c - kPieces);
+            }
+        });
+        for (int i = i0 + tid; i < i1; i += kThreads)
+            S.pend_score[(size_t)bg * S.P + pend_fill + i] = a.cand_score[(size_t)(b * n + i) * G + g];
+    }
     __threadfence();
+    __syncthreads();
     if (tid == 0) {
         const unsigned old = atomicAdd(S.tickets + bg, 1u);
         *tail_flag = (int)old == 2 * ntiles - 1;
@@ -583,26 +644,20 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*tail_flag == 0) return;
 
-    // ---------------- last CTA of (b, g): commit the block, then the forced admit ----------------
+    // ---------------- last CTA of (b, g): the ring write, then the forced admit ----------------
     __threadfence();
-    const bool fits = pend_fill + n <= S.P;
-    constexpr int kPieces = kRowBytes / 16;   // 32 per row
-    for (int e = tid; e < n * kPieces; e += kThreads) {
-        const int i = e / kPieces, c = e % kPieces;
+    copy_pieces<kThreads, 16>(n * 2 * kPieces, [&](int e, const uint4*& from_p, uint4*& to_p) {
+        const int i = e / (2 * kPieces), c = e % (2 * kPieces);
         const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
-        const int slot = (s + i) % S.R;
-        const size_t dst = ((size_t)bg * S.R + slot) * kHeadDim;
-        reinterpret_cast<uint4*>(S.ring_k + dst)[c] = reinterpret_cast<const uint4*>(a.k + src)[c];
-        reinterpret_cast<uint4*>(S.ring_v + dst)[c] = reinterpret_cast<const uint4*>(a.v + src)[c];
-        if (fits) {
-            const size_t pd = ((size_t)bg * S.P + pend_fill + i) * kHeadDim;
-            reinterpret_cast<uint4*>(S.pend_k + pd)[c] = reinterpret_cast<const uint4*>(a.cand_k + src)[c];
-            reinterpret_cast<uint4*>(S.pend_v + pd)[c] = reinterpret_cast<const uint4*>(a.cand_v + src)[c];
+        const size_t dst = ((size_t)bg * S.R + (s + i) % S.R) * kHeadDim;
+        if (c < kPieces) {
+            from_p = reinterpret_cast<const uint4*>(a.k + src) + c;
+            to_p = reinterpret_cast<uint4*>(S.ring_k + dst) + c;
+        } else {
+            from_p = reinterpret_cast<const uint4*>(a.v + src) + (c - kPieces);
+            to_p = reinterpret_cast<uint4*>(S.ring_v + dst) + (c - kPieces);
         }
-    }
-    if (fits)
-        for (int i = tid; i < n; i += kThreads)
-            S.pend_score[(size_t)bg * S.P + pend_fill + i] = a.cand_score[(size_t)(b * n + i) * G + g];
+    });
     const int np = fits ? pend_fill + n : pend_fill;
     __syncthreads();
     if (tid == 0) {
