@@ -77,11 +77,12 @@ constexpr int kSmemW = kSmemXch + 4096;               // w_g rows of the group's
 constexpr int kSmemBytes = kSmemW + 4096 + 1024;      // + 1 KiB for alignment
 constexpr int kXchEndM = 128, kXchEndL = 512, kXchGate = 768;
 constexpr int kSoftmaxThreads = 256;                  // warps 0-7
-// warp 8: TMA producer; warp 9: Q K^T issuer (even CTA) or stale-row cleaner (odd CTA);
-// warp 10: P V issuer (even CTA).  Two issuing warps keep the tensor pipe fed while either
-// one waits on a barrier.
-constexpr int kWarpTma = 8, kWarpQK = 9, kWarpPV = 10;
-constexpr int kThreads = 352;
+// warp 8: TMA producer; warps 9 and 11: Q K^T issuers for even and odd chunks (even CTA;
+// in the odd CTA warp 9 is the stale-row cleaner); warp 10: P V issuer (even CTA).  The
+// tensor pipe queues few instructions, so it idles whenever its only issuer waits on a
+// barrier; three issuing warps keep it fed while any one of them waits.
+constexpr int kWarpTma = 8, kWarpQK = 9, kWarpPV = 10, kWarpQK2 = 11;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
 constexpr int kTilesPerCluster = 2;
@@ -259,14 +260,14 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             for (int jj = max(0, nchunks - kStages); jj < nchunks; ++jj)
                 if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
                     break;
-        } else if (warp == kWarpQK) {
-            // ---------------- even CTA: Q K^T issuer ----------------
+        } else if (warp == kWarpQK || (warp == kWarpQK2 && pr == 0)) {
+            // ---------------- even CTA: Q K^T issuers (warp 9: even chunks, warp 11: odd) ----------------
             // S of chunk j lives in columns kColS0 / kColS1 by j & 1 and P in shared memory, so
             // Q K^T of chunk j + 2 may start as soon as the softmax group has read S of chunk j.
             constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(2 * kRows, kChunk, false, false);
             bool ok = ptx::mbar_wait_warp(&bars[kQReady], 0, abort_flag, S.status);
             ptx::tc_fence_after();
-            for (int j = 0; ok && j < nchunks; ++j) {
+            for (int j = warp == kWarpQK ? 0 : 1; ok && j < nchunks; j += 2) {
                 if (j >= 2) {
                     ok = ptx::mbar_wait_warp(&bars[kSFree + (j & 1)], ((j - 2) >> 1) & 1, abort_flag, S.status);
                     if (!ok) break;
