@@ -99,10 +99,11 @@ __device__ __forceinline__ int admit_block_scan(int v, int* warp_tot, int* total
 }
 
 // Admit group bg of layer view s with nb committed records and np candidates
-// (both already validated).  Every thread of the CTA (NT of them) must call it;
+// (both already validated).  Every thread of the CTA (NT of them) must call it; each
+// thread keeps U 16-byte pieces of the row copies in flight;
 // `scratch` is shared memory of admit_scratch_bytes(A, P) bytes, 16-aligned.
 // Writes the bank rows, scores and the counters bank_fill and pend_fill.
-template <int NT>
+template <int NT, int U = 8>
 __device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t* scratch) {
     const int A = s.A, P = s.P;
     const int tid = threadIdx.x;
@@ -243,7 +244,7 @@ __device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t*
     uint4* bk = reinterpret_cast<uint4*>(s.bank_k + (size_t)bg * A * kHeadDim);
     uint4* bv = reinterpret_cast<uint4*>(s.bank_v + (size_t)bg * A * kHeadDim);
     constexpr int kChunks = kRowBytes / 16;   // 32 per row
-    copy_pieces<NT, 8>(n_adm * 2 * kChunks, [&](int e, const uint4*& from_p, uint4*& to_p) {
+    copy_pieces<NT, U>(n_adm * 2 * kChunks, [&](int e, const uint4*& from_p, uint4*& to_p) {
         const int j = e / (2 * kChunks);
         const int c = e % (2 * kChunks);
         const int from = src[j], to = dest[j];

@@ -581,19 +581,17 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::bulk_commit();
     }
     if (warp < 8) {
-        // 4 threads per row, 64 dims each
-        const int crow = 64 * phase + (tid >> 2), qd = tid & 3;
-        const int ctok = kTileTok * T + (crow >> 2), chead = g * kQPerGroup + (crow & 3);
-        const size_t qoff = ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim + 64 * qd;
-        const float gate = xch[kXchGate + crow];
+        // one row per warp at a time: lane L makes output dims [8 L, 8 L + 8) (16 contiguous bytes)
         const bool got = ptx::mbar_wait_warp(&bars[kXfer], 0, abort_flag, S.status);
-        const uint8_t* prow = smem + 128 * 1024 + (size_t)(crow - 64 * phase) * 1024;
-        const uint8_t* mrow = smem + (size_t)crow * 1024;
-        uint4* orow = reinterpret_cast<uint4*>(a.out + qoff);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t off0 = (uint32_t)(((16 * qd + 2 * e) ^ (crow & 7)) << 4);
-            const uint32_t off1 = (uint32_t)(((16 * qd + 2 * e + 1) ^ (crow & 7)) << 4);
+#pragma unroll 2
+        for (int rr = 0; rr < 8; ++rr) {
+            const int lrow = 8 * warp + rr, crow = 64 * phase + lrow;
+            const int ctok = kTileTok * T + (crow >> 2), chead = g * kQPerGroup + (crow & 3);
+            const float gate = xch[kXchGate + crow];
+            const uint32_t off0 = (uint32_t)(((2 * lane) ^ (crow & 7)) << 4);
+            const uint32_t off1 = (uint32_t)(((2 * lane + 1) ^ (crow & 7)) << 4);
+            const uint8_t* mrow = smem + (size_t)crow * 1024;
+            const uint8_t* prow = smem + 128 * 1024 + (size_t)lrow * 1024;
             const float4 m0 = *reinterpret_cast<const float4*>(mrow + off0);
             const float4 m1 = *reinterpret_cast<const float4*>(mrow + off1);
             float4 t0 = make_float4(0.f, 0.f, 0.f, 0.f), t1 = t0;
@@ -608,14 +606,45 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             r.y = pack_bf16(l0.z + gate * c0.z, l0.w + gate * c0.w);
             r.z = pack_bf16(l1.x + gate * c1.x, l1.y + gate * c1.y);
             r.w = pack_bf16(l1.z + gate * c1.z, l1.w + gate * c1.w);
-            orow[e] = r;
+            reinterpret_cast<uint4*>(a.out + ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim)[lane] = r;
         }
     }
     if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
 
+    // Ring write.  The slot of block token i holds position s + i - R, which queries up to token i
+    // still read, so the rows of local pair p (tokens [64 p, 64 p + 64)) may be written once local
+    // pairs 0..p have finished reading the ring.  Each local pair's even CTA marks its pair done in
+    // bits 8.. of the group's ticket word and writes the rows of every pair its mark completes the
+    // prefix for (the count of finished CTAs is in bits 0..7).
+    if (phase == 0 && pr == 0) {
+        int* range = tail_flag + 1;
+        if (tid == 0) {
+            __threadfence();
+            const unsigned bit = 1u << (8 + (blockIdx.x >> 2));
+            const unsigned old = atomicOr(S.tickets + bg, bit) >> 8;
+            __threadfence();
+            range[0] = __ffs(~old) - 1;            // pairs done in a row before this mark
+            range[1] = __ffs(~(old | (bit >> 8))) - 1;   // and after it
+        }
+        __syncthreads();
+        const int t0 = min(n, 2 * kTileTok * range[0]), t1 = min(n, 2 * kTileTok * range[1]);
+        copy_pieces<kThreads, 8>((t1 - t0) * 2 * kRowBytes / 16, [&](int e, const uint4*& from_p, uint4*& to_p) {
+            constexpr int kP = kRowBytes / 16;
+            const int i = t0 + e / (2 * kP), c = e % (2 * kP);
+            const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
+            const size_t dst = ((size_t)bg * S.R + (s + i) % S.R) * kHeadDim;
+            if (c < kP) {
+                from_p = reinterpret_cast<const uint4*>(a.k + src) + c;
+                to_p = reinterpret_cast<uint4*>(S.ring_k + dst) + c;
+            } else {
+                from_p = reinterpret_cast<const uint4*>(a.v + src) + (c - kP);
+                to_p = reinterpret_cast<uint4*>(S.ring_v + dst) + (c - kP);
+            }
+        });
+    }
+
     // This CTA's share of the candidates goes to pending now (nothing in this launch reads those
-    // slots before the last CTA's admit); the ring write has to wait until every CTA of the group
-    // has read the ring.
+    // slots before the last CTA's admit).
     const bool fits = pend_fill + n <= S.P;
     constexpr int kPieces = kRowBytes / 16;   // 32 per row
     const int nct = gridDim.x, share = (n + nct - 1) / nct;
@@ -640,25 +669,13 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (tid == 0) {
         const unsigned old = atomicAdd(S.tickets + bg, 1u);
-        *tail_flag = (int)old == 2 * ntiles - 1;
+        *tail_flag = (int)(old & 0xFFu) == 2 * ntiles - 1;
     }
     __syncthreads();
     if (*tail_flag == 0) return;
 
-    // ---------------- last CTA of (b, g): the ring write, then the forced admit ----------------
+    // ---------------- last CTA of (b, g): the forced admit ----------------
     __threadfence();
-    copy_pieces<kThreads, 16>(n * 2 * kPieces, [&](int e, const uint4*& from_p, uint4*& to_p) {
-        const int i = e / (2 * kPieces), c = e % (2 * kPieces);
-        const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
-        const size_t dst = ((size_t)bg * S.R + (s + i) % S.R) * kHeadDim;
-        if (c < kPieces) {
-            from_p = reinterpret_cast<const uint4*>(a.k + src) + c;
-            to_p = reinterpret_cast<uint4*>(S.ring_k + dst) + c;
-        } else {
-            from_p = reinterpret_cast<const uint4*>(a.v + src) + (c - kPieces);
-            to_p = reinterpret_cast<uint4*>(S.ring_v + dst) + (c - kPieces);
-        }
-    });
     const int np = fits ? pend_fill + n : pend_fill;
     __syncthreads();
     if (tid == 0) {
@@ -667,7 +684,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         c[2] = np;
         if (!fits) atomicOr(S.status, (unsigned)RMA_STATUS_PREFILL_PENDING_OVERFLOW);
     }
-    if (np > 0) admit_group<kThreads>(S, bg, bank_fill, np, smem);
+    if (np > 0) admit_group<kThreads, 16>(S, bg, bank_fill, np, smem);
     if (tid == 0) S.tickets[bg] = 0u;
 }
 
