@@ -40,6 +40,7 @@ UNIT = "tokens/s"
 BYTES_FULL = 4 * 1023 * 1024 + 4 * 1024 * 1024 + 8192 + 8192 + 4096 + 4096
 FALLBACK_HBM_GBS = 6650.0
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "rma_decode_batch512.md")
+PREFILL_PROFILE = os.path.join(ROOT, "profiles", "rma_prefill_block.md")
 
 
 def log(*a):
@@ -60,11 +61,11 @@ def kernel_source_hash(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic(profile_path: str, source: str):
+def profiled_traffic(profile_path: str, source: str, key: str = "traffic_bytes_per_launch_batch512"):
     """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source.
 
-    The summary holds a line 'traffic_bytes_per_launch_batch512: <int>' and a
-    line 'kernel_source_sha256_16: <hash>'; a different hash means the kernel
+    The summary holds a line '<key>: <int>' and a line
+    'kernel_source_sha256_16: <hash>'; a different hash means the kernel
     changed since the counters were taken, and traffic is reported as null.
     """
     if not os.path.exists(profile_path):
@@ -78,7 +79,7 @@ def profiled_traffic(profile_path: str, source: str):
     if vals.get("kernel_source_sha256_16") != kernel_source_hash(source):
         return None
     try:
-        return int(vals["traffic_bytes_per_launch_batch512"])
+        return int(vals[key])
     except (KeyError, ValueError):
         return None
 
@@ -337,17 +338,21 @@ def run_prefill(args) -> None:
     peak = float(pk["bf16_tflops_sustained"])
     achieved = total_flops / (sum(call_ms) / 1e3) / 1e12
     line = {
-        "metric": "RMA block-prefill TFLOP/s (algorithmic), batch 8 x 8 layers x 128 blocks of 256",
+        "metric": f"RMA block-prefill TFLOP/s (algorithmic), batch {B} x {L} layers x {blocks} blocks of {n}",
         "value": total_flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "tokens_per_s": B * n * blocks / (ms / 1e3),
         "n_gpus": 1, "steps": blocks, "ms_total": ms, "higher_is_better": True, "dtype": "bf16",
         "accumulate": "f32", "data": "synthetic",
         "config": {"workload": f"block prefill: {B} sequences x {L} RMA layers, {blocks} blocks of {n} queries "
                                "from an empty state; each block attends causally to the 1024-position window and "
                                "to the bank committed before it, then admits its 256 candidates",
-                   "algorithmic_tflop": total_flops / 1e12},
+                   "algorithmic_tflop": total_flops / 1e12,
+                   "l2": f"inputs larger than L2: the {st.buffer.numel() / 1e6:.0f} MB state spans {L} layers and each call "
+                         "reads another layer's ring and bank"},
         "clocks": clocks,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(PREFILL_PROFILE, "rma_prefill.cu", "traffic_bytes_per_launch_prefill"),
+                     "traffic_note": "one steady-state launch (ring and bank full), profiles/rma_prefill_block.md",
                      "kernel": "rma_prefill_block (one launch: attention, commit, forced admit)",
                      "call_ms_mean": sum(call_ms) / len(call_ms),
                      "peak_source": "measured bf16_tflops_sustained (MEASURED_PEAKS.json)"},
