@@ -15,6 +15,13 @@ Usage:
   torchrun --nproc-per-node N bench.py --gpus N ...     (one replica per GPU)
   python bench.py --workload long|ragged|prefill         (other workloads)
 
+Other workloads: "long" = 1 sequence at pos 131,072 (full ring and bank), its
+8-layer steps replayed from CUDA graphs, reported with per-step latency median
+and p99; "ragged" = random ring/bank/pending fills with 16-level scores
+(--batch 32..512); "prefill" = 8 sequences x 8 layers, blocks of 256 from an
+empty state, in TFLOP/s.  Roofline bytes always come from the exact fills of
+every timed launch.
+
 Multi-GPU: sequences are independent, so each rank runs its own 512-sequence
 replica with no data-path collective ("weak" scaling); the only collectives
 are the harness's barrier and the max-over-ranks of the timed duration.
@@ -411,21 +418,68 @@ def main():
     out = torch.empty(B, 16, 256, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step(i, ev=None):
+    def step(i, ev=None, strm=None):
+        strm = strm if strm is not None else stream
         for l in range(L):
             x = pool[i % 16][l]
             if ev is not None:
-                ev[l][0].record(stream)
+                ev[l][0].record(strm)
             rma.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"], x["cand_score"],
-                            w[l], b[l], out, ws, stream=stream)
+                            w[l], b[l], out, ws, stream=strm)
             if ev is not None:
-                ev[l][1].record(stream)
+                ev[l][1].record(strm)
+
+    # algorithmic bytes of every launch, from the counters the steps will see (tracked on the host
+    # with the method's counter rules: ring fill min(pos, R), the admit at pending == P)
+    cnt0 = st.counters.cpu().numpy().astype("int64")
+    pos, bank, pend = cnt0[..., 0].copy(), cnt0[..., 1].copy(), cnt0[..., 2].copy()
+
+    def launch_bytes(l):
+        return int(((pos[l].clip(max=1023) + bank[l]) * 1024).sum() + B * 24576)
+
+    def advance(l):
+        pos[l] += 1
+        pend[l] += 1
+        full = pend[l] == 256
+        bank[l] = (bank[l] + 256 * full).clip(max=1024)
+        pend[l][full] = 0
+
+    def step_bytes():
+        tot = 0
+        for l in range(L):
+            tot += launch_bytes(l)
+            advance(l)
+        return tot
+
+    # the long-context case is launch-latency bound: its 8 launches per step are replayed from
+    # CUDA graphs (one per input set) instead of being issued one by one from Python
+    graphs = None
+    if kind == "long":
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(stream)
+        with torch.cuda.stream(cs):
+            step(0, strm=cs)
+        cs.synchronize()
+        graphs = []
+        for sidx in range(16):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cs):
+                step(sidx, strm=cs)
+            graphs.append(gr)
+        torch.cuda.synchronize(device)
+        st.counters.copy_(torch.from_numpy(cnt0).to(torch.int32))   # the captured steps ran nothing
+        torch.cuda.synchronize(device)
 
     for i in range(args.warmup):
-        step(i)
+        if graphs is not None:
+            graphs[i % 16].replay()
+        else:
+            step(i)
+        step_bytes()
     K = args.steps
     evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
            for _ in range(K)]
+    timed_bytes = []
     t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = None
     try:
@@ -440,7 +494,13 @@ def main():
     torch.cuda.synchronize(device)
     t0e.record(stream)
     for i in range(K):
-        step(args.warmup + i, evs[i])
+        if graphs is not None:
+            evs[i][0][0].record(stream)
+            graphs[(args.warmup + i) % 16].replay()
+            evs[i][0][1].record(stream)
+        else:
+            step(args.warmup + i, evs[i])
+        timed_bytes.append(step_bytes())
     t1e.record(stream)
     torch.cuda.synchronize(device)
     if world > 1:
@@ -454,13 +514,18 @@ def main():
     ms_per_step = ms / K
     value = world * B * K / (ms / 1e3)
 
-    # dominant kernel: rma_decode, per-launch duration from the events around each launch
-    durs = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
-    dec_ms = sum(durs) / len(durs)
-    if kind == "batch":
-        alg_bytes = B * BYTES_FULL
+    # dominant kernel: rma_decode, per-launch duration from the events around each launch (for
+    # the graph-replayed long-context steps: the step time over its 8 launches)
+    latency = None
+    if graphs is not None:
+        step_ms = sorted(evs[i][0][0].elapsed_time(evs[i][0][1]) for i in range(K))
+        dec_ms = sum(step_ms) / len(step_ms) / L
+        latency = {"unit": "us per 8-layer step (CUDA graph replay)", "median": 1e3 * step_ms[len(step_ms) // 2],
+                   "p99": 1e3 * step_ms[min(len(step_ms) - 1, int(0.99 * len(step_ms)))], "min": 1e3 * step_ms[0]}
     else:
-        alg_bytes = None
+        durs = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
+        dec_ms = sum(durs) / len(durs)
+    alg_bytes = sum(timed_bytes) / (K * L)     # per launch, from the exact per-step fills
     peak, peak_kind = peaks()
 
     # end to end through the public API: host (pinned) inputs in, host output out, every step
@@ -536,11 +601,16 @@ def main():
                          "traffic": profiled_traffic(DECODE_PROFILE, "rma_decode.cu") if kind == "batch" else None,
                          "kernel": "rma_decode (decode_kernel)", "kernel_ms": dec_ms,
                          "algorithmic_bytes_per_launch": alg_bytes,
+                         "algorithmic_bytes_note": "ring min(pos, 1023) + bank_fill rows x 1 KiB per group, plus "
+                                                   "q, out, current K/V and the ring write, from the exact fills of "
+                                                   "every timed launch",
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                          else "fallback 6.65 TB/s"},
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        if latency is not None:
+            line["latency"] = latency
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

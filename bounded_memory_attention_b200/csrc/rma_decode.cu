@@ -335,6 +335,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     float* misc = coef + (kMaxSplits + 1) * 4;                                             // scur[4], gate[4]
     const uint16_t* kc = a.k_cur + (size_t)bg * kHeadDim;
     const uint16_t* vc = a.v_cur + (size_t)bg * kHeadDim;
+    const float* parts = a.ws + (size_t)bg * n_splits * kPartialFloats;
+    // every split's maxima and sums (8 floats each) into shared memory in one L2 round trip
+    // (the pipeline region is free now)
+    float* pml = reinterpret_cast<float*>(smem);   // [n_splits][8]
+    for (int i = tid; i < n_splits * 8; i += kThreads)
+        pml[i] = __ldcg(parts + (size_t)(i >> 3) * kPartialFloats + (i & 7));
     if (warp < 4) {
         // s_cur[h] = scale * log2(e) * q_h . k_cur
         const int h = warp;
@@ -360,36 +366,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     }
     __syncthreads();
 
-    const float* parts = a.ws + (size_t)bg * n_splits * kPartialFloats;
     if (tid < 8) {
         const int h = tid & 3;
         if (tid < 4) {
             // local softmax: ring splits plus the current token
             const float scur = misc[h];
             float M = scur;
-            for (int sp = 0; sp < a.ring_splits; ++sp) M = fmaxf(M, __ldcg(parts + sp * kPartialFloats + h));
+            for (int sp = 0; sp < a.ring_splits; ++sp) M = fmaxf(M, pml[sp * 8 + h]);
             float L = fast_ex2(scur - M);
-            for (int sp = 0; sp < a.ring_splits; ++sp) {
-                const float* pp = parts + sp * kPartialFloats;
-                L += fast_ex2(__ldcg(pp + h) - M) * __ldcg(pp + 4 + h);
-            }
+            for (int sp = 0; sp < a.ring_splits; ++sp) L += fast_ex2(pml[sp * 8 + h] - M) * pml[sp * 8 + 4 + h];
             const float inv = 1.f / L;
-            for (int sp = 0; sp < a.ring_splits; ++sp)
-                coef[sp * 4 + h] = fast_ex2(__ldcg(parts + sp * kPartialFloats + h) - M) * inv;
+            for (int sp = 0; sp < a.ring_splits; ++sp) coef[sp * 4 + h] = fast_ex2(pml[sp * 8 + h] - M) * inv;
             coef[n_splits * 4 + h] = fast_ex2(scur - M) * inv;
         } else {
             // anchor softmax over the bank splits, scaled by the gate
             float M = -CUDART_INF_F;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp) M = fmaxf(M, __ldcg(parts + sp * kPartialFloats + h));
+            for (int sp = a.ring_splits; sp < n_splits; ++sp) M = fmaxf(M, pml[sp * 8 + h]);
             float L = 0.f;
             const float Mu = (M == -CUDART_INF_F) ? 0.f : M;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp) {
-                const float* pp = parts + sp * kPartialFloats;
-                L += fast_ex2(__ldcg(pp + h) - Mu) * __ldcg(pp + 4 + h);
-            }
+            for (int sp = a.ring_splits; sp < n_splits; ++sp) L += fast_ex2(pml[sp * 8 + h] - Mu) * pml[sp * 8 + 4 + h];
             const float scale = (L > 0.f) ? misc[4 + h] / L : 0.f;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp)
-                coef[sp * 4 + h] = fast_ex2(__ldcg(parts + sp * kPartialFloats + h) - Mu) * scale;
+            for (int sp = a.ring_splits; sp < n_splits; ++sp) coef[sp * 4 + h] = fast_ex2(pml[sp * 8 + h] - Mu) * scale;
         }
     }
     __syncthreads();
@@ -401,9 +398,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         const uint2 vr = *reinterpret_cast<const uint2*>(vc + d);
         const float2 va = bf2_to_f2(vr.x), vb = bf2_to_f2(vr.y);
         float4 o = make_float4(cc * va.x, cc * va.y, cc * vb.x, cc * vb.y);
-        for (int sp = 0; sp < n_splits; ++sp) {
+        // the splits' accumulators, sixteen loads in flight at a time (same summation order)
+        const float* pacc = parts + 8 + h * kHeadDim + d;
+        int sp = 0;
+        for (; sp + 16 <= n_splits; sp += 16) {
+            float4 v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(pacc + (size_t)(sp + u) * kPartialFloats));
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float c = coef[(sp + u) * 4 + h];
+                o.x += c * v[u].x; o.y += c * v[u].y; o.z += c * v[u].z; o.w += c * v[u].w;
+            }
+        }
+        for (; sp < n_splits; ++sp) {
             const float c = coef[sp * 4 + h];
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(parts + sp * kPartialFloats + 8 + h * kHeadDim + d));
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pacc + (size_t)sp * kPartialFloats));
             o.x += c * v.x; o.y += c * v.y; o.z += c * v.z; o.w += c * v.w;
         }
         const __nv_bfloat162 o01 = __floats2bfloat162_rn(o.x, o.y);
