@@ -91,6 +91,23 @@ def profiled_traffic(profile_path: str, source: str, key: str = "traffic_bytes_p
         return None
 
 
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank calls it with its own device-timed duration
+    (the identity for one process)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi clock and throttle-reason samples while the timed region runs."""
 
@@ -506,13 +523,9 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t0e.elapsed_time(t1e)
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0e.elapsed_time(t1e), world, device)
     ms_per_step = ms / K
-    value = world * B * K / (ms / 1e3)
+    value = whole_job_rate(world, B * K, ms)
 
     # dominant kernel: rma_decode, per-launch duration from the events around each launch (for
     # the graph-replayed long-context steps: the step time over its 8 launches)
@@ -559,12 +572,8 @@ def main():
             e2e_step(i)
         a1.record(stream)
         torch.cuda.synchronize(device)
-        ems = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([ems], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * B * Ke / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        ems = max_over_ranks(a0.elapsed_time(a1), world, device)
+        e2e = {"value": whole_job_rate(world, B * Ke, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": Ke,
                "path": "pinned host inputs -> device copies -> rma_decode_step x 8 layers -> "
                        "pinned host outputs, one stream"}
