@@ -167,19 +167,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         vbase = a.s.bank_v + off;
     }
 
-    // ---- q of the group's 4 heads, this lane's 8 dims, in the log2 domain ----
-    float2 q2[kQPerGroup][4];
-    const uint16_t* qg = a.q + ((size_t)b * G * kQPerGroup + (size_t)g * kQPerGroup) * kHeadDim;
-#pragma unroll
-    for (int h = 0; h < kQPerGroup; ++h) {
-        const uint4 r = ld_nc_v4(qg + h * kHeadDim + lane * 8);
-        const float2 s2 = make_float2(a.qscale, a.qscale);
-        q2[h][0] = __fmul2_rn(bf2_to_f2(r.x), s2);
-        q2[h][1] = __fmul2_rn(bf2_to_f2(r.y), s2);
-        q2[h][2] = __fmul2_rn(bf2_to_f2(r.z), s2);
-        q2[h][3] = __fmul2_rn(bf2_to_f2(r.w), s2);
-    }
-
     // ---- per-warp cp.async pipeline over this warp's tiles ----
     uint8_t* wsm = smem + warp * (kStages * kStageBytes);
     const uint32_t wsm_a = smem_addr(wsm);
@@ -205,6 +192,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         if (s < my_n) issue(s, s);
         cp_commit();
     }
+
+    // ---- q of the group's 4 heads, this lane's 8 dims, in the log2 domain (loaded while the
+    //      first K/V tiles are in flight) ----
+    float2 q2[kQPerGroup][4];
+    const uint16_t* qg = a.q + ((size_t)b * G * kQPerGroup + (size_t)g * kQPerGroup) * kHeadDim;
+#pragma unroll
+    for (int h = 0; h < kQPerGroup; ++h) {
+        const uint4 r = ld_nc_v4(qg + h * kHeadDim + lane * 8);
+        const float2 s2 = make_float2(a.qscale, a.qscale);
+        q2[h][0] = __fmul2_rn(bf2_to_f2(r.x), s2);
+        q2[h][1] = __fmul2_rn(bf2_to_f2(r.y), s2);
+        q2[h][2] = __fmul2_rn(bf2_to_f2(r.z), s2);
+        q2[h][3] = __fmul2_rn(bf2_to_f2(r.w), s2);
+    }
+
 
     float m_run = -CUDART_INF_F, l_run = 0.f;
     float2 acc[kQPerGroup][4];
