@@ -20,28 +20,33 @@
 // keys, so each CTA loads only half of every 64-key K/V chunk (K rows split
 // by key, V split by dimension), which halves the K/V bytes per FLOP.
 //   * tensor memory (512 columns, the pair allocates together): O [0,256)
-//     FP32, S/P double buffer [256,320) and [320,384), Q [384,512) packed
-//     BF16 (Q K^T takes A from tensor memory; shared memory holds a six-stage
-//     ring of K/V half-chunks);
+//     FP32, S double buffer [256,320) and [320,384) (chunk j in S_(j & 1)),
+//     Q [384,512) packed BF16 (Q K^T takes A from tensor memory); shared
+//     memory holds a five-stage ring of K/V half-chunks and one BF16 P buffer
+//     per softmax group (the UMMA K-major layout, 128-byte swizzle);
 //   * warp 8 of each CTA loads its half of each chunk with TMA (128B swizzle);
-//   * warp 9 of the even CTA issues S = Q K^T (N 64, K 256) and O += P V
-//     (N 256, K 64, P from tensor memory, V an MN-major operand) and commits
-//     to the barriers of both CTAs; warp 9 of the odd CTA checks its half
-//     landed, clears stale V rows and signals the even CTA;
+//   * in the even CTA, warps 9 and 11 issue S = Q K^T (N 64, K 256) for even
+//     and odd chunks and warp 10 issues O += P V (N 256, K 64, P and V from
+//     shared memory, V an MN-major operand), committing to the barriers of both
+//     CTAs; the tensor pipe queues few instructions, and three issuers keep it
+//     fed while any one waits.  Warp 9 of the odd CTA checks its half landed,
+//     clears stale V rows and signals the even CTA;
 //   * warps 0-7 of each CTA are the softmax for its own rows: two
-//     warpgroups, each thread one row and half of the chunk's keys; they load
-//     Q into tensor memory, read S, mask by position (whole halves that are
-//     all visible or all hidden skip the per-key test), exchange the row max
-//     through shared memory, keep the online max / sum in FP32 (moving the
-//     reference max only when it grows by more than 2^8), write BF16 P over
-//     S, and finally normalise O.
-// Tail: every CTA writes its normalised rows into its own shared memory; after
-// a cluster barrier the local and anchor CTAs of a tile each combine half of
-// its rows, reading the other result through distributed shared memory:
-// out = local + gate * anchor in FP32, rounded once to BF16.  A per-(sequence,
-// group) ticket finds the last CTA, which writes the block into the ring and
-// the pending buffer (every read of the block is over by then) and runs the
-// forced admit.  No load is multicast: every CTA reads its own data.
+//     warpgroups that take alternate chunks, each thread a whole 64-key row;
+//     they load Q into tensor memory (and compute the gate), read S, release
+//     its columns for Q K^T of chunk j + 2, mask by position (32-key halves
+//     that are all visible skip the per-key test), hand the reference max from
+//     chunk to chunk through shared memory (moving it only when a chunk's max
+//     exceeds it by more than 2^8, then rescaling O), write P to shared memory,
+//     keep one row sum per group and finally normalise O.
+// Tail: every CTA writes its normalised rows into its own shared memory and
+// pushes the 64 rows the other CTA of its tile (local <-> anchor) combines into
+// that CTA's free stage area with one bulk copy (no multicast); each combines
+// its half: out = local + gate * anchor in FP32, rounded once to BF16.  Each CTA
+// appends its share of the candidates to pending; local pairs write the block's
+// K/V into the ring as soon as every earlier pair has finished reading it; the
+// last CTA of the (sequence, group) runs the forced admit.  No load is
+// multicast: every CTA reads its own data.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
