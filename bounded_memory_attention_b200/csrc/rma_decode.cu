@@ -76,6 +76,12 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     return r;
 }
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -338,71 +344,89 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     const uint16_t* kc = a.k_cur + (size_t)bg * kHeadDim;
     const uint16_t* vc = a.v_cur + (size_t)bg * kHeadDim;
     const float* parts = a.ws + (size_t)bg * n_splits * kPartialFloats;
-    // every split's maxima and sums (8 floats each) into shared memory in one L2 round trip
-    // (the pipeline region is free now)
+    // Every load the merge needs is issued before any of its results is used, so that the
+    // merging CTA pays one L2 round trip instead of a chain of them: this thread's q / k_cur /
+    // w_g pieces, every split's maxima and sums (into shared memory; the pipeline region is
+    // free now) and the first 16 splits' accumulators for its 4 output dims.
+    const int oh = tid >> 6, od = (tid & 63) * 4;          // this thread's output head and dims
+    const float* pacc = parts + 8 + oh * kHeadDim + od;
+    float4 pre[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+        if (u < n_splits) pre[u] = __ldcg(reinterpret_cast<const float4*>(pacc + (size_t)u * kPartialFloats));
+    const int mh = warp & 3;                                // this warp's head for s_cur / gate
+    const int head = g * kQPerGroup + mh;
+    const uint4 qr = ld_nc_v4(qg + mh * kHeadDim + lane * 8);
+    uint4 kr = make_uint4(0, 0, 0, 0);
+    float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+    if (warp < 4) {
+        kr = ld_nc_v4(kc + lane * 8);
+    } else {
+        w0 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + lane * 8));
+        w1 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + lane * 8 + 4));
+    }
     float* pml = reinterpret_cast<float*>(smem);   // [n_splits][8]
     for (int i = tid; i < n_splits * 8; i += kThreads)
         pml[i] = __ldcg(parts + (size_t)(i >> 3) * kPartialFloats + (i & 7));
     if (warp < 4) {
         // s_cur[h] = scale * log2(e) * q_h . k_cur
-        const int h = warp;
-        const uint4 kr = ld_nc_v4(kc + lane * 8);
-        const uint4 qr = ld_nc_v4(qg + h * kHeadDim + lane * 8);
         const float2 s2 = make_float2(a.qscale, a.qscale);
         const float2 qh[4] = {__fmul2_rn(bf2_to_f2(qr.x), s2), __fmul2_rn(bf2_to_f2(qr.y), s2),
                               __fmul2_rn(bf2_to_f2(qr.z), s2), __fmul2_rn(bf2_to_f2(qr.w), s2)};
-        const float s = warp_sum(dot8(qh, kr));
-        if (lane == 0) misc[h] = s;
+        const float sc = warp_sum(dot8(qh, kr));
+        if (lane == 0) misc[mh] = sc;
     } else {
         // gate[h] = tanh(q_h . w_g[head] + b_g[head]), with the unscaled query
-        const int h = warp - 4;
-        const int head = g * kQPerGroup + h;
-        const uint4 qr = ld_nc_v4(qg + h * kHeadDim + lane * 8);
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + lane * 8));
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim + lane * 8 + 4));
         const float2 q0 = bf2_to_f2(qr.x), q1 = bf2_to_f2(qr.y), qq2 = bf2_to_f2(qr.z), q3 = bf2_to_f2(qr.w);
-        float d = q0.x * w0.x + q0.y * w0.y + q1.x * w0.z + q1.y * w0.w +
-                  qq2.x * w1.x + qq2.y * w1.y + q3.x * w1.z + q3.y * w1.w;
-        d = warp_sum(d);
-        if (lane == 0) misc[4 + h] = tanhf(d + a.b_g[head]);
+        float dg = q0.x * w0.x + q0.y * w0.y + q1.x * w0.z + q1.y * w0.w +
+                   qq2.x * w1.x + qq2.y * w1.y + q3.x * w1.z + q3.y * w1.w;
+        dg = warp_sum(dg);
+        if (lane == 0) misc[4 + mh] = tanhf(dg + a.b_g[head]);
     }
     __syncthreads();
 
-    if (tid < 8) {
-        const int h = tid & 3;
-        if (tid < 4) {
-            // local softmax: ring splits plus the current token
-            const float scur = misc[h];
-            float M = scur;
-            for (int sp = 0; sp < a.ring_splits; ++sp) M = fmaxf(M, pml[sp * 8 + h]);
-            float L = fast_ex2(scur - M);
-            for (int sp = 0; sp < a.ring_splits; ++sp) L += fast_ex2(pml[sp * 8 + h] - M) * pml[sp * 8 + 4 + h];
-            const float inv = 1.f / L;
-            for (int sp = 0; sp < a.ring_splits; ++sp) coef[sp * 4 + h] = fast_ex2(pml[sp * 8 + h] - M) * inv;
-            coef[n_splits * 4 + h] = fast_ex2(scur - M) * inv;
+    // Coefficients: warp w takes head w & 3 of the local softmax (ring splits and the current
+    // token, w < 4) or of the anchor softmax (bank splits, scaled by the gate, w >= 4); its
+    // lanes take the splits.
+    {
+        const int h = warp & 3;
+        const bool local = warp < 4;
+        const int sp0 = local ? 0 : a.ring_splits, sp1 = local ? a.ring_splits : n_splits;
+        const float scur = misc[h];
+        float M = local ? scur : -CUDART_INF_F;
+        for (int sp = sp0 + lane; sp < sp1; sp += 32) M = fmaxf(M, pml[sp * 8 + h]);
+        M = warp_max(M);
+        const float Mu = (M == -CUDART_INF_F) ? 0.f : M;
+        float L = 0.f;
+        for (int sp = sp0 + lane; sp < sp1; sp += 32) L += fast_ex2(pml[sp * 8 + h] - Mu) * pml[sp * 8 + 4 + h];
+        L = warp_sum(L);
+        float scale;
+        if (local) {
+            L += fast_ex2(scur - Mu);
+            scale = 1.f / L;
         } else {
-            // anchor softmax over the bank splits, scaled by the gate
-            float M = -CUDART_INF_F;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp) M = fmaxf(M, pml[sp * 8 + h]);
-            float L = 0.f;
-            const float Mu = (M == -CUDART_INF_F) ? 0.f : M;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp) L += fast_ex2(pml[sp * 8 + h] - Mu) * pml[sp * 8 + 4 + h];
-            const float scale = (L > 0.f) ? misc[4 + h] / L : 0.f;
-            for (int sp = a.ring_splits; sp < n_splits; ++sp) coef[sp * 4 + h] = fast_ex2(pml[sp * 8 + h] - Mu) * scale;
+            scale = (L > 0.f) ? misc[4 + h] / L : 0.f;
         }
+        for (int sp = sp0 + lane; sp < sp1; sp += 32) coef[sp * 4 + h] = fast_ex2(pml[sp * 8 + h] - Mu) * scale;
+        if (local && lane == 0) coef[n_splits * 4 + h] = fast_ex2(scur - Mu) * scale;
     }
     __syncthreads();
 
     {
-        const int h = tid >> 6;
-        const int d = (tid & 63) * 4;
+        const int h = oh, d = od;
         const float cc = coef[n_splits * 4 + h];
         const uint2 vr = *reinterpret_cast<const uint2*>(vc + d);
         const float2 va = bf2_to_f2(vr.x), vb = bf2_to_f2(vr.y);
         float4 o = make_float4(cc * va.x, cc * va.y, cc * vb.x, cc * vb.y);
-        // the splits' accumulators, sixteen loads in flight at a time (same summation order)
-        const float* pacc = parts + 8 + h * kHeadDim + d;
-        int sp = 0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            if (u < n_splits) {
+                const float c = coef[u * 4 + h];
+                o.x += c * pre[u].x; o.y += c * pre[u].y; o.z += c * pre[u].z; o.w += c * pre[u].w;
+            }
+        }
+        // the remaining splits' accumulators, sixteen loads in flight at a time (same summation order)
+        int sp = 16;
         for (; sp + 16 <= n_splits; sp += 16) {
             float4 v[16];
 #pragma unroll
@@ -423,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         uint2 packed;
         packed.x = *reinterpret_cast<const uint32_t*>(&o01);
         packed.y = *reinterpret_cast<const uint32_t*>(&o23);
-        const int head = g * kQPerGroup + h;
-        *reinterpret_cast<uint2*>(a.out + ((size_t)b * G * kQPerGroup + head) * kHeadDim + d) = packed;
+        const int ohead = g * kQPerGroup + h;
+        *reinterpret_cast<uint2*>(a.out + ((size_t)b * G * kQPerGroup + ohead) * kHeadDim + d) = packed;
     }
 
     // ---- state writes: every split of (b, g) has finished reading ----
