@@ -229,7 +229,45 @@ def cpu_oracle_decode(n_seq: int, n_layers: int, n_steps: int, seed: int = 0) ->
         dt = time.perf_counter() - t0
     return {"value": n_seq * n_steps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n_seq} of the 512 sequences x {n_layers} layers x {n_steps} steps "
-                      f"(decode + admit), FP64 numpy oracle, 1 thread; {dt:.1f} s"}
+                      f"(decode + admit), FP64 numpy oracle, 1 thread; {dt:.1f} s", "cpu": host_cpu()}
+
+
+def host_cpu() -> str:
+    """The host CPU's model name and logical core count."""
+    model = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{model}, {os.cpu_count()} logical cores"
+
+
+def cpu_oracle_prefill(seed: int = 0) -> dict:
+    """Time the oracle on steady-state prefill blocks (ring and bank full) of one sequence at one
+    layer, in algorithmic GFLOP/s (one host thread)."""
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(batch=1, n_layers=1)
+    cont = si.state_contents(1, 1, 4, 256, 1023, 1024, 256, seed=seed)
+    st = oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, pos=4096, bank_fill=1024, pend_fill=0)
+    w, b = si.gate_params(1, 16, 256, seed)
+    n_blocks = 16
+    xs = [{k: _np(v) for k, v in si.prefill_inputs(1, 256, 4, 4, 256, seed=seed + j).items()} for j in range(n_blocks)]
+    flops = prefill_flops(1, 1, 256, 20)[-1] * n_blocks   # blocks at steady state
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for x in xs:
+            oracle.prefill_block(st, 0, x["q"], x["k"], x["v"], x["cand_k"], x["cand_v"], x["cand_score"],
+                                 w[0].numpy(), b[0].numpy())
+        dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e9, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_blocks} blocks of 256 tokens x 1 sequence x 1 layer (ring and bank full, forced "
+                      f"admits), FP64 numpy oracle, 1 thread; {dt:.1f} s", "cpu": host_cpu()}
 
 
 def run_reference(args) -> None:
@@ -382,6 +420,12 @@ def run_prefill(args) -> None:
                      "peak_source": "measured bf16_tflops_sustained (MEASURED_PEAKS.json)"},
         "gpu_launches": blocks * L,
     }
+    if not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = cpu_oracle_prefill()
+        except Exception as ex:   # a report, never a reason to lose the bench line
+            line["cpu_baseline"] = {"value": None, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"failed: {ex}"}
     print(json.dumps(line), flush=True)
 
 
