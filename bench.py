@@ -590,37 +590,67 @@ def main():
     if not args.no_e2e:
         h2d, d2h = step_input_bytes(B, L)
         host_in = [[{k: v.cpu().pin_memory() for k, v in pool[s][l].items()} for l in range(L)] for s in range(4)]
-        host_out = torch.empty(L, B, 16, 256, dtype=torch.bfloat16).pin_memory()
-        dev_in = [{k: torch.empty_like(v, device=device) for k, v in host_in[0][l].items()} for l in range(L)]
-        outs = torch.empty(L, B, 16, 256, dtype=torch.bfloat16, device=device)
+        # two sets of device inputs and outputs, so that the copies of one step overlap the
+        # kernels of the next: inputs go up on one copy stream, results come down on another
+        host_out = [torch.empty(L, B, 16, 256, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        dev_in = [[{k: torch.empty_like(v, device=device) for k, v in host_in[0][l].items()} for l in range(L)]
+                  for _ in range(2)]
+        outs = [torch.empty(L, B, 16, 256, dtype=torch.bfloat16, device=device) for _ in range(2)]
+        up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        read = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step(i):
-            for l in range(L):
-                for k, v in host_in[i % 4][l].items():
-                    dev_in[l][k].copy_(v, non_blocking=True)
-            for l in range(L):
-                x = dev_in[l]
-                rma.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"], x["cand_score"],
-                                w[l], b[l], outs[l], ws, stream=stream)
-            host_out.copy_(outs, non_blocking=True)
+        def e2e_run(n_steps):
+            up.wait_stream(stream)
+            down.wait_stream(stream)
+
+            def h2d_of(i):
+                k = i % 2
+                if i >= 2:
+                    up.wait_event(done[k])              # step i - 2 no longer reads these inputs
+                with torch.cuda.stream(up):
+                    for l in range(L):
+                        for name, v in host_in[i % 4][l].items():
+                            dev_in[k][l][name].copy_(v, non_blocking=True)
+                in_ready[k].record(up)
+
+            h2d_of(0)
+            for i in range(n_steps):
+                k = i % 2
+                if i + 1 < n_steps:
+                    h2d_of(i + 1)
+                stream.wait_event(in_ready[k])
+                if i >= 2:
+                    stream.wait_event(read[k])          # step i - 2's results have come down
+                for l in range(L):
+                    x = dev_in[k][l]
+                    rma.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"],
+                                    x["cand_score"], w[l], b[l], outs[k][l], ws, stream=stream)
+                done[k].record(stream)
+                down.wait_event(done[k])
+                with torch.cuda.stream(down):
+                    host_out[k].copy_(outs[k], non_blocking=True)
+                read[k].record(down)
+            stream.wait_stream(up)
+            stream.wait_stream(down)
 
         Ke = max(16, K // 8)
-        for i in range(3):
-            e2e_step(i)
+        e2e_run(3)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(device)
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for i in range(Ke):
-            e2e_step(i)
+        e2e_run(Ke)
         a1.record(stream)
         torch.cuda.synchronize(device)
         ems = max_over_ranks(a0.elapsed_time(a1), world, device)
         e2e = {"value": whole_job_rate(world, B * Ke, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": Ke,
-               "path": "pinned host inputs -> device copies -> rma_decode_step x 8 layers -> "
-                       "pinned host outputs, one stream"}
+               "path": "pinned host inputs -> device copies (copy stream) -> rma_decode_step x 8 layers -> "
+                       "pinned host outputs (second copy stream); two buffer sets, so the copies of one "
+                       "step overlap the kernels of the next"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and kind == "batch":
