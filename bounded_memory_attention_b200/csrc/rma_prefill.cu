@@ -617,22 +617,23 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
 
     // Ring write.  The slot of block token i holds position s + i - R, which queries up to token i
-    // still read, so the rows of local pair p (tokens [64 p, 64 p + 64)) may be written once local
-    // pairs 0..p have finished reading the ring.  Each local pair's even CTA marks its pair done in
-    // bits 8.. of the group's ticket word and writes the rows of every pair its mark completes the
-    // prefix for (the count of finished CTAs is in bits 0..7).
-    if (phase == 0 && pr == 0) {
+    // still read, so the rows of tile T (tokens [32 T, 32 T + 32)) may be written once tiles 0..T
+    // have finished reading the ring; both CTAs of a local pair are done here (the cluster barrier
+    // above follows every MMA of the pair).  Each local CTA marks its tile in bits 8.. of the
+    // group's ticket word and writes the rows of every tile its mark completes the prefix for (the
+    // count of finished CTAs is in bits 0..7).
+    if (phase == 0) {
         int* range = tail_flag + 1;
         if (tid == 0) {
             __threadfence();
-            const unsigned bit = 1u << (8 + (blockIdx.x >> 2));
+            const unsigned bit = 1u << (8 + T);
             const unsigned old = atomicOr(S.tickets + bg, bit) >> 8;
             __threadfence();
-            range[0] = __ffs(~old) - 1;            // pairs done in a row before this mark
+            range[0] = __ffs(~old) - 1;            // tiles done in a row before this mark
             range[1] = __ffs(~(old | (bit >> 8))) - 1;   // and after it
         }
         __syncthreads();
-        const int t0 = min(n, 2 * kTileTok * range[0]), t1 = min(n, 2 * kTileTok * range[1]);
+        const int t0 = min(n, kTileTok * range[0]), t1 = min(n, kTileTok * range[1]);
         copy_pieces<kThreads, 8>((t1 - t0) * 2 * kRowBytes / 16, [&](int e, const uint4*& from_p, uint4*& to_p) {
             constexpr int kP = kRowBytes / 16;
             const int i = t0 + e / (2 * kP), c = e % (2 * kP);
