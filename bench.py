@@ -91,6 +91,40 @@ def profiled_traffic(profile_path: str, source: str, key: str = "traffic_bytes_p
         return None
 
 
+class FillTracker:
+    """Algorithmic bytes of every decode launch, from the state's counters tracked on the host
+    with the method's counter rules: the step reads min(pos, R) ring rows and bank_fill bank rows
+    of every group (1 KiB each, K and V), then pos += 1, pend_fill += 1, and a group whose
+    pending buffer fills is admitted (bank_fill = min(A, bank_fill + P), pend_fill = 0).
+    Fixed bytes per sequence: q 8,192 + out 8,192 + current K/V 4,096 + ring write 4,096."""
+
+    FIXED = 8192 + 8192 + 4096 + 4096
+
+    def __init__(self, counters, R: int = 1023, A: int = 1024, P: int = 256):
+        c = counters.astype("int64")
+        self.pos, self.bank, self.pend = c[..., 0].copy(), c[..., 1].copy(), c[..., 2].copy()
+        self.R, self.A, self.P = R, A, P
+
+    def launch_bytes(self, layer: int) -> int:
+        rows = self.pos[layer].clip(max=self.R) + self.bank[layer]
+        return int(rows.sum() * 1024 + self.pos.shape[1] * self.FIXED)
+
+    def advance(self, layer: int) -> None:
+        self.pos[layer] += 1
+        self.pend[layer] += 1
+        full = self.pend[layer] == self.P
+        self.bank[layer] = (self.bank[layer] + self.P * full).clip(max=self.A)
+        self.pend[layer][full] = 0
+
+    def step_bytes(self) -> int:
+        """Bytes of one step over every layer, then the counters advance."""
+        tot = 0
+        for layer in range(self.pos.shape[0]):
+            tot += self.launch_bytes(layer)
+            self.advance(layer)
+        return tot
+
+
 def max_over_ranks(ms: float, world: int, device=None) -> float:
     """The slowest rank's time: every rank calls it with its own device-timed duration
     (the identity for one process)."""
@@ -490,27 +524,10 @@ def main():
             if ev is not None:
                 ev[l][1].record(strm)
 
-    # algorithmic bytes of every launch, from the counters the steps will see (tracked on the host
-    # with the method's counter rules: ring fill min(pos, R), the admit at pending == P)
+    # algorithmic bytes of every launch, from the counters the steps will see
     cnt0 = st.counters.cpu().numpy().astype("int64")
-    pos, bank, pend = cnt0[..., 0].copy(), cnt0[..., 1].copy(), cnt0[..., 2].copy()
-
-    def launch_bytes(l):
-        return int(((pos[l].clip(max=1023) + bank[l]) * 1024).sum() + B * 24576)
-
-    def advance(l):
-        pos[l] += 1
-        pend[l] += 1
-        full = pend[l] == 256
-        bank[l] = (bank[l] + 256 * full).clip(max=1024)
-        pend[l][full] = 0
-
-    def step_bytes():
-        tot = 0
-        for l in range(L):
-            tot += launch_bytes(l)
-            advance(l)
-        return tot
+    fills = FillTracker(cnt0)
+    step_bytes = fills.step_bytes
 
     # the long-context case is launch-latency bound: its 8 launches per step are replayed from
     # CUDA graphs (one per input set) instead of being issued one by one from Python
