@@ -1,7 +1,7 @@
 """CPU oracle for the RMA attention hot path (test infrastructure only).
 
 Only the test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
-leg may import this package.  The CUDA library never calls it.
+and reference legs may import this package.  The CUDA library never calls it.
 """
 from .rma_oracle import *  # noqa: F401,F403
 from .rma_oracle import (Config, State, new_state, state_from_arrays, copy_state, decode_step, admit,

@@ -1,8 +1,8 @@
 """CPU oracle for the Rock Memory Anchors (RMA) attention hot path.
 
 TEST INFRASTRUCTURE.  This module exists to check the CUDA library.  Only the
-test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import it.  The product path (the C-ABI library and its
+test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference (``--impl reference``) legs may import it.  The product path (the C-ABI library and its
 Python binding) never calls it and has no CPU fallback.
 
 It is a plain, slow, step-by-step restatement of what the pages say the RMA
