@@ -21,11 +21,8 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// One CTA per (b, g).  prefill_n > 0: first account for a prefill block of
-// prefill_n tokens whose K/V and candidates were already written (pos += n;
-// pend_fill += n if the candidates fit, else RMA_STATUS_PREFILL_PENDING_OVERFLOW).
-__global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__ LayerView s, int force,
-                                                         int prefill_n) {
+// One CTA per (b, g).
+__global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__ LayerView s, int force) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int g = blockIdx.x, b = blockIdx.y;
     const int bg = b * s.G + g;
@@ -38,23 +35,13 @@ __global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__
         nb = min(max(nb, 0), s.A);
         np = min(max(np, 0), s.P);
     }
-    if (prefill_n > 0) {
-        const bool fits = np + prefill_n <= s.P;
-        __syncthreads();   // every thread has read the counters
-        if (tid == 0) {
-            cnt[0] = max(cnt[0], 0) + prefill_n;
-            if (fits) cnt[2] = np + prefill_n;
-            else atomicOr(s.status, (unsigned)RMA_STATUS_PREFILL_PENDING_OVERFLOW);
-        }
-        if (fits) np += prefill_n;
-    }
     if (!(np == s.P || (force && np > 0))) return;
     admit_group<kThreads>(s, bg, nb, np, smem);
 }
 
 }  // namespace
 
-cudaError_t launch_admit(const LayerView& s, int force, int prefill_n, cudaStream_t stream) {
+cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream) {
     const size_t smem = admit_scratch_bytes(s.A, s.P);
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
@@ -63,7 +50,7 @@ cudaError_t launch_admit(const LayerView& s, int force, int prefill_n, cudaStrea
         configured = smem;
     }
     dim3 grid(s.G, s.B);
-    admit_kernel<<<grid, kThreads, smem, stream>>>(s, force, prefill_n);
+    admit_kernel<<<grid, kThreads, smem, stream>>>(s, force);
     return cudaGetLastError();
 }
 

@@ -189,16 +189,16 @@ void rma_state_free(rma_state* st) { delete as_state(st); }
 int rma_workspace_bytes(const rma_state* st, int n_tok, size_t* out) {
     if (!st || !out) return fail(RMA_ERR_INVALID_ARG, "state and out must be non-NULL");
     const State* s = as_state(st);
-    if (n_tok == 1) {
+    if (n_tok < 1) return fail(RMA_ERR_INVALID_ARG, "n_tok must be >= 1");
+    if (n_tok > kMaxPrefillTokens) return fail(RMA_ERR_UNSUPPORTED, "n_tok > 256");
+    size_t bytes = prefill_workspace_bytes(s->cfg, n_tok);
+    if (n_tok == 1) {   // a decode step, or a one-token prefill block: enough for either
         const Splits sp = decode_splits(*s);
-        *out = (size_t)s->cfg.batch * s->cfg.n_groups * (sp.ring_splits + sp.bank_splits) * kPartialFloats * 4;
-        return RMA_OK;
+        const size_t dec = (size_t)s->cfg.batch * s->cfg.n_groups * (sp.ring_splits + sp.bank_splits) * kPartialFloats * 4;
+        bytes = dec > bytes ? dec : bytes;
     }
-    if (n_tok == s->cfg.pend_slots) {
-        *out = prefill_workspace_bytes(s->cfg, n_tok);
-        return RMA_OK;
-    }
-    return fail(RMA_ERR_INVALID_ARG, "n_tok must be 1 (decode) or pend_slots (prefill)");
+    *out = bytes;
+    return RMA_OK;
 }
 
 int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_splits) {
@@ -281,7 +281,7 @@ int rma_admit(rma_state* st, int layer, int force, void* stream) {
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;
     if (force != 0 && force != 1) return fail(RMA_ERR_INVALID_ARG, "force must be 0 or 1");
-    cudaError_t e = launch_admit(layer_view(*s, layer), force, 0, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_admit(layer_view(*s, layer), force, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_admit");
     return RMA_OK;
 }
@@ -298,9 +298,9 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
     for (const void* p : a16)
         if (!aligned(p, 16)) return fail(RMA_ERR_MISALIGNED, "q, k, v, cand_k, cand_v, w_g, out, ws need 16-byte alignment");
     if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
-    if (n_tok != s->cfg.pend_slots || n_tok % 64 != 0 || n_tok > 256 || n_tok > s->cfg.ring_slots)
-        return fail(RMA_ERR_UNSUPPORTED,
-                    "this build needs n_tok == pend_slots, a multiple of 64, at most 256 and at most ring_slots");
+    if (n_tok < 1) return fail(RMA_ERR_INVALID_ARG, "n_tok must be >= 1");
+    if (n_tok > kMaxPrefillTokens || n_tok > s->cfg.ring_slots)
+        return fail(RMA_ERR_UNSUPPORTED, "this build needs n_tok <= 256 and n_tok <= ring_slots");
     if (ws_bytes < prefill_workspace_bytes(s->cfg, n_tok))
         return fail(RMA_ERR_BUFFER_TOO_SMALL, "workspace smaller than rma_workspace_bytes(st, n_tok)");
     PrefillArgs a;

@@ -83,8 +83,9 @@ cudaError_t static_decode_scratch(void** ptr);
 
 // Launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
-// prefill_n > 0: also advance pos and pend_fill for a prefill block of that many tokens.
-cudaError_t launch_admit(const LayerView& s, int force, int prefill_n, cudaStream_t stream);
+cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream);
+// Longest prefill block (tokens per sequence) one rma_prefill_block call takes.
+constexpr int kMaxPrefillTokens = 256;
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok);
 

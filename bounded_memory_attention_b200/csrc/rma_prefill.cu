@@ -15,6 +15,9 @@
 // the bank (phase 1).  Four CTAs form a thread-block cluster:
 //   rank 0: tile 2p, local     rank 1: tile 2p+1, local
 //   rank 2: tile 2p, anchor    rank 3: tile 2p+1, anchor
+// A block may hold any n from 1 to 256 tokens: the grid covers ceil(n / 64)
+// pairs of tiles, rows past the last token repeat its query and are not
+// stored, and keys past it are masked (their V rows cleared).
 // Ranks (0,1) and (2,3) are CTA pairs for the 2-SM tensor-core MMA
 // (tcgen05 cta_group::2, M = 256): both tiles of a pair read exactly the same
 // keys, so each CTA loads only half of every 64-key K/V chunk (K rows split
@@ -330,8 +333,10 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
             {
                 // this half of the Q row -> tensor memory columns [384 + 64 wg, +64) as packed BF16
+                // (rows past the block's last token repeat its query; their results are not stored)
                 const uint4* qrow =
-                    reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + tok) * HQ + head) * kHeadDim) + 16 * wg;
+                    reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + min(tok, n - 1)) * HQ + head) * kHeadDim) +
+                    16 * wg;
                 uint32_t r0[32], r1[32];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -611,7 +616,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             r.y = pack_bf16(l0.z + gate * c0.z, l0.w + gate * c0.w);
             r.z = pack_bf16(l1.x + gate * c1.x, l1.y + gate * c1.y);
             r.w = pack_bf16(l1.z + gate * c1.z, l1.w + gate * c1.w);
-            reinterpret_cast<uint4*>(a.out + ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim)[lane] = r;
+            if (ctok < n) reinterpret_cast<uint4*>(a.out + ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim)[lane] = r;
         }
     }
     if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
@@ -741,9 +746,10 @@ size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok) {
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const LayerView& s = a.s;
     const int B = s.B, G = s.G, n = a.n_tok;
-    // tiles come in pairs (64 tokens); the ticket counts 2 * ntiles arrivals
-    if (n % (kTilesPerCluster * kTileTok) != 0 || n > 256 || n > s.R) return cudaErrorNotSupported;
-    const int ntiles = n / kTileTok;
+    // tiles come in pairs (64 tokens, the last one possibly ragged); the ticket counts 2 * ntiles
+    // arrivals in 8 bits and marks one bit per tile in bits 8..15
+    if (n < 1 || n > kMaxPrefillTokens || n > s.R) return cudaErrorNotSupported;
+    const int ntiles = kTilesPerCluster * ((n + kTilesPerCluster * kTileTok - 1) / (kTilesPerCluster * kTileTok));
     Tmaps tm;
     const uint64_t row = (uint64_t)kHeadDim * 2;
     bool ok = make_map(&tm.k, a.k, G, (uint64_t)B * n, row, row * G, 1, kHalfKeys) &&

@@ -130,9 +130,11 @@ RMA_API int rma_state_layout(const rma_state* st, rma_layout* out);
 RMA_API void rma_state_free(rma_state* st);
 
 /* Workspace (device scratch, 256-byte aligned) a call with n_tok tokens per
- * sequence needs: n_tok == 1 for rma_decode_step, n_tok == pend_slots for
- * rma_prefill_block.  The caller owns it; its contents need not be preserved
- * between calls, but two calls in flight at once need two workspaces. */
+ * sequence needs: n_tok == 1 for rma_decode_step (the size also covers a
+ * one-token prefill block), 1 <= n_tok <= 256 for rma_prefill_block.
+ * RMA_ERR_INVALID_ARG for n_tok < 1, RMA_ERR_UNSUPPORTED above 256.  The
+ * caller owns it; its contents need not be preserved between calls, but two
+ * calls in flight at once need two workspaces. */
 RMA_API int rma_workspace_bytes(const rma_state* st, int n_tok, size_t* out);
 
 /* Decode split-K shape: the ring and the bank are each cut into this many
@@ -229,9 +231,11 @@ RMA_API int rma_admit(rma_state* st, int layer, int force, void* stream);
  *   out         bf16 [batch][n_tok][n_groups*q_per_group][head_dim]  (written)
  *   ws          workspace of rma_workspace_bytes(st, n_tok) bytes
  * One launch: the admit runs inside it once every read of the block is done.
- * This build requires n_tok == pend_slots, n_tok a multiple of 64, at most
- * 256 and at most ring_slots (RMA_ERR_UNSUPPORTED otherwise).  Alignment as
- * in rma_decode_step. */
+ * n_tok is any length from 1 (RMA_ERR_INVALID_ARG below) to 256 and at most
+ * ring_slots (RMA_ERR_UNSUPPORTED above): a prompt whose length is not a
+ * multiple of pend_slots ends in a shorter block, and a block may follow
+ * decode steps (pend_fill != 0 at its start).  Alignment as in
+ * rma_decode_step. */
 RMA_API int rma_prefill_block(rma_state* st, int layer, int n_tok,
                       const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,

@@ -5,6 +5,8 @@
   * a block of n = P tokens starting with an empty pending buffer equals n
     decode steps (each followed by the admit rule): same outputs, same state
     bytes; this ties prefill to the brute-force-pinned decode;
+  * a block of any n <= P tokens that starts with pend_fill != 0 (its
+    candidates fit) equals n decode steps followed by a forced admit;
   * check (d): records admitted at the end of block k are invisible to block
     k's queries and visible to block k+1's;
   * g = +-1/2: anchor part equals brute force over the bank as committed
@@ -45,9 +47,9 @@ def _args(x):
     return [x[k] for k in ("q", "k", "v", "cand_k", "cand_v", "cand_score")]
 
 
-@pytest.mark.parametrize("ring_slots,n", [(7, 4), (3, 4), (5, 5), (9, 2)])
-def test_gate_zero_equals_causal_window_bruteforce(ring_slots, n):
-    cfg = _cfg(ring_slots=ring_slots, pend_slots=n)
+@pytest.mark.parametrize("ring_slots,n,pend_slots", [(7, 4, 4), (3, 4, 4), (5, 5, 5), (9, 2, 2), (7, 3, 8)])
+def test_gate_zero_equals_causal_window_bruteforce(ring_slots, n, pend_slots):
+    cfg = _cfg(ring_slots=ring_slots, pend_slots=pend_slots)
     st = _state(cfg, seed=1, bank_fill=3)
     w = np.zeros((cfg.n_q_heads, cfg.head_dim), np.float32)
     bg = np.zeros(cfg.n_q_heads, np.float32)
@@ -55,7 +57,7 @@ def test_gate_zero_equals_causal_window_bruteforce(ring_slots, n):
     hist_v = [[[] for _ in range(cfg.n_groups)] for _ in range(cfg.batch)]
     R = cfg.ring_slots
     for blk in range(6):
-        x = _block(cfg, 100 + blk)
+        x = _block(cfg, 100 + blk, n=n)
         s0 = st.pos.copy()
         _, out = oracle.prefill_block(st, 0, *_args(x), w, bg, return_f64=True)
         for b in range(cfg.batch):
@@ -92,6 +94,30 @@ def test_block_equals_decode_steps():
         for name in ("ring_k", "ring_v", "bank_k", "bank_v", "bank_score", "pend_k", "pend_v", "pend_score",
                      "pos", "bank_fill", "pend_fill"):
             assert np.array_equal(getattr(st_p, name), getattr(st_d, name)), name
+
+
+@pytest.mark.parametrize("n,pend0", [(1, 0), (3, 2), (5, 0), (6, 2), (8, 0)])
+def test_ragged_block_equals_decode_steps_then_forced_admit(n, pend0):
+    """Blocks shorter than P, after decode steps left candidates pending: the block's reads and
+    writes are those of n decode steps, and its forced admit is the admit at the end."""
+    cfg = _cfg(ring_slots=7, pend_slots=8)
+    st_p = _state(cfg, seed=12, bank_fill=4, pend_fill=pend0, pos=9)
+    st_d = oracle.copy_state(st_p)
+    w = si.f32_normal((cfg.n_q_heads, cfg.head_dim), 13, std=0.2).numpy()
+    bg = si.f32_normal((cfg.n_q_heads,), 14, std=0.2).numpy()
+    for blk in range(3):
+        x = _block(cfg, 300 + blk, n=n)
+        _, out_p = oracle.prefill_block(st_p, 0, *_args(x), w, bg, return_f64=True)
+        for i in range(n):
+            _, out_d = oracle.decode_step(st_d, 0, x["q"][:, i], x["k"][:, i], x["v"][:, i], x["cand_k"][:, i],
+                                          x["cand_v"][:, i], x["cand_score"][:, i], w, bg, return_f64=True)
+            oracle.admit(st_d, 0)
+            np.testing.assert_allclose(out_p[:, i], out_d, rtol=1e-12, atol=1e-13)
+        oracle.admit(st_d, 0, force=True)
+        for name in ("ring_k", "ring_v", "bank_k", "bank_v", "bank_score", "pend_k", "pend_v", "pend_score",
+                     "pos", "bank_fill", "pend_fill"):
+            assert np.array_equal(getattr(st_p, name), getattr(st_d, name)), name
+        assert int(st_p.pend_fill.max()) == 0 and st_p.status == 0
 
 
 def test_block_admits_are_invisible_to_own_block_and_visible_to_next():
