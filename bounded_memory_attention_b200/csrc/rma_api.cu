@@ -37,7 +37,7 @@ int check_config(const rma_config* c) {
     if (!(std::isfinite(c->softmax_scale) && c->softmax_scale > 0.f))
         return fail(RMA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     if (c->q_per_group != kQPerGroup || c->head_dim != kHeadDim)
-        return fail(RMA_ERR_UNSUPPORTED, "this build implements q_per_group == 4 and head_dim == 256");
+        return fail(RMA_ERR_UNSUPPORTED, "the library implements q_per_group == 4 and head_dim == 256");
     if (c->ring_slots > (1 << 20)) return fail(RMA_ERR_UNSUPPORTED, "ring_slots > 2^20");
     if (c->bank_slots + c->pend_slots > 4096) return fail(RMA_ERR_UNSUPPORTED, "bank_slots + pend_slots > 4096");
     if (c->batch > 65535 || c->n_groups > 65535) return fail(RMA_ERR_UNSUPPORTED, "batch or n_groups > 65535");
@@ -300,7 +300,7 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
     if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
     if (n_tok < 1) return fail(RMA_ERR_INVALID_ARG, "n_tok must be >= 1");
     if (n_tok > kMaxPrefillTokens || n_tok > s->cfg.ring_slots)
-        return fail(RMA_ERR_UNSUPPORTED, "this build needs n_tok <= 256 and n_tok <= ring_slots");
+        return fail(RMA_ERR_UNSUPPORTED, "rma_prefill_block takes n_tok <= 256 and n_tok <= ring_slots");
     if (ws_bytes < prefill_workspace_bytes(s->cfg, n_tok))
         return fail(RMA_ERR_BUFFER_TOO_SMALL, "workspace smaller than rma_workspace_bytes(st, n_tok)");
     PrefillArgs a;

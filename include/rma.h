@@ -53,7 +53,7 @@ extern "C" {
 /* ---- return codes ---- */
 #define RMA_OK                    0
 #define RMA_ERR_INVALID_ARG      -1  /* null pointer, bad layer index, bad flag value */
-#define RMA_ERR_UNSUPPORTED      -2  /* a shape this build does not implement */
+#define RMA_ERR_UNSUPPORTED      -2  /* a shape the library does not implement */
 #define RMA_ERR_BUFFER_TOO_SMALL -3  /* state buffer or workspace smaller than required */
 #define RMA_ERR_CUDA             -4  /* a CUDA runtime call or kernel launch failed */
 #define RMA_ERR_MISALIGNED       -5  /* a pointer lacks the alignment stated below */
@@ -76,7 +76,7 @@ extern "C" {
  * not valid.  Indicates a fault in the library, never an input condition. */
 #define RMA_STATUS_TIMEOUT                  16u
 
-/* Dimensions.  This build implements q_per_group == 4 and head_dim == 256
+/* Dimensions.  The library implements q_per_group == 4 and head_dim == 256
  * (RMA_ERR_UNSUPPORTED otherwise), any n_groups >= 1, ring_slots in
  * [1, 1<<20], bank_slots >= 1, pend_slots >= 1, bank_slots + pend_slots <= 4096. */
 typedef struct rma_config {
