@@ -13,14 +13,15 @@ larger than L2, so no flush is needed between steps.
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   torchrun --nproc-per-node N bench.py --gpus N ...     (one replica per GPU)
-  python bench.py --workload long|ragged|prefill         (other workloads)
+  python bench.py --workload long|ragged|prefill|admit   (other workloads)
 
 Other workloads: "long" = 1 sequence at pos 131,072 (full ring and bank), its
 8-layer steps replayed from CUDA graphs, reported with per-step latency median
 and p99; "ragged" = random ring/bank/pending fills with 16-level scores
 (--batch 32..512); "prefill" = 8 sequences x 8 layers, blocks of 256 from an
-empty state, in TFLOP/s.  Roofline bytes always come from the exact fills of
-every timed launch.
+empty state, in TFLOP/s; "admit" = the standalone admit of a batch whose
+sequences are in phase (every bank and every pending buffer full), in GB/s.
+Roofline bytes always come from the exact fills of every timed launch.
 
 Multi-GPU: sequences are independent, so each rank runs its own 512-sequence
 replica with no data-path collective ("weak" scaling); the only collectives
@@ -48,6 +49,13 @@ BYTES_FULL = 4 * 1023 * 1024 + 4 * 1024 * 1024 + 8192 + 8192 + 4096 + 4096
 FALLBACK_HBM_GBS = 6650.0
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "rma_decode_batch512.md")
 PREFILL_PROFILE = os.path.join(ROOT, "profiles", "rma_prefill_block.md")
+ADMIT_PROFILE = os.path.join(ROOT, "profiles", "rma_admit_batch512.md")
+ADMIT_SOURCES = ("rma_admit.cu", "rma_admit_impl.cuh")
+# algorithmic bytes of one group's admit: the 1,024 + 256 scores read once, then for every
+# admitted candidate its K and V rows (1 KiB together) read from pending and written to the
+# bank, and its score written (the two counters written are left out)
+ADMIT_SCORE_BYTES = (1024 + 256) * 4
+ADMIT_ROW_BYTES = 2 * 1024 + 4
 
 
 def log(*a):
@@ -63,9 +71,14 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash(name: str) -> str:
-    with open(os.path.join(ROOT, "bounded_memory_attention_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_source_hash(name) -> str:
+    """First 16 hex digits of the SHA-256 of a kernel's source file (or, for a tuple of names,
+    of the files' contents concatenated in that order)."""
+    h = hashlib.sha256()
+    for n in ((name,) if isinstance(name, str) else name):
+        with open(os.path.join(ROOT, "bounded_memory_attention_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(profile_path: str, source: str, key: str = "traffic_bytes_per_launch_batch512"):
@@ -463,6 +476,138 @@ def run_prefill(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def admitted_counts(bank_score, pend_score):
+    """How many candidates each group admits when every bank slot and every pending slot is
+    filled: those among the first A of the A + P records ordered by score (descending), then
+    committed before candidate, then slot (ascending).  bank_score [..., A] and pend_score
+    [..., P] float32 without NaN -> int array [...].  Byte counting for the roofline only."""
+    import numpy as np
+    A, P = bank_score.shape[-1], pend_score.shape[-1]
+    lead = bank_score.shape[:-1]
+    sc = np.concatenate([bank_score.reshape(-1, A), pend_score.reshape(-1, P)], axis=1)
+    cand = np.broadcast_to(np.r_[np.zeros(A, np.int8), np.ones(P, np.int8)], sc.shape)
+    slot = np.broadcast_to(np.r_[np.arange(A), np.arange(P)], sc.shape)
+    order = np.lexsort((slot, cand, -sc), axis=-1)       # -0.0 and +0.0 compare equal, as in the order
+    return np.take_along_axis(cand, order[:, :A], axis=1).sum(axis=1).reshape(lead)
+
+
+def cpu_oracle_admit(seed: int = 0, n_seq: int = 32, reps: int = 16) -> dict:
+    """Time the oracle's admit on groups with every bank and pending slot filled (scores ~ N(0,1)),
+    in algorithmic GB/s (one host thread); each repetition starts from a fresh copy of the state."""
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(batch=n_seq, n_layers=1)
+    cont = si.state_contents(1, n_seq, 4, 256, 1023, 1024, 256, seed=seed)
+    st0 = oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, pos=131_072, bank_fill=1024,
+                                   pend_fill=256)
+    n_adm = admitted_counts(st0.bank_score, st0.pend_score)
+    nbytes = n_seq * 4 * ADMIT_SCORE_BYTES + ADMIT_ROW_BYTES * int(n_adm.sum())
+    dt = 0.0
+    with threadpool_limits(limits=1):
+        for _ in range(reps):
+            st = oracle.copy_state(st0)
+            t0 = time.perf_counter()
+            oracle.admit(st, 0)
+            dt += time.perf_counter() - t0
+    return {"value": reps * nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} admits of {n_seq} sequences x 4 groups (one layer, every bank and pending "
+                      f"slot filled), FP64/numpy oracle, 1 thread; {dt:.1f} s", "cpu": host_cpu()}
+
+
+def run_admit(args) -> None:
+    """The standalone admit of a batch whose sequences are in phase: every group's bank (1,024)
+    and pending buffer (256) full, scores ~ N(0,1).  One step = rma_admit for each layer.  Before
+    each step the bank scores and the counters are restored (untimed), so every step makes the
+    same selection; the K/V rows the previous step copied stay, which changes no byte count."""
+    import torch
+    from bounded_memory_attention_b200 import build
+    build.build()
+    import bounded_memory_attention_b200 as rma
+    device = torch.device("cuda", 0)
+    B, L, G = args.batch or 512, args.layers or 8, 4
+    st = rma.State(rma.Config(batch=B, n_layers=L), device=device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(0)
+    for name in ("bank_k", "bank_v", "pend_k", "pend_v"):
+        getattr(st, name).normal_(generator=gen)
+    st.bank_score.normal_(generator=gen)
+    st.pend_score.normal_(generator=gen)
+    score0 = st.bank_score.clone()
+    cnt0 = torch.zeros(L, B, G, 4, dtype=torch.int32, device=device)
+    cnt0[..., 0], cnt0[..., 1], cnt0[..., 2] = 131_072, 1024, 256
+    n_adm = admitted_counts(score0.cpu().numpy(), st.pend_score.cpu().numpy())   # [L, B, G]
+    launch_bytes = [B * G * ADMIT_SCORE_BYTES + ADMIT_ROW_BYTES * int(n_adm[l].sum()) for l in range(L)]
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        st.bank_score.copy_(score0)
+        st.counters.copy_(cnt0)
+        for l in range(L):
+            if ev is not None:
+                ev[l][0].record(stream)
+            rma.admit(st, l, stream=stream)          # runs where pending is full: every group
+            if ev is not None:
+                ev[l][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    # the bookkeeping above must describe what the kernel did: one changed score per admitted candidate
+    changed = (st.bank_score != score0).sum(dim=-1).cpu().numpy()
+    counts_agree = bool((changed == n_adm).all())
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+           for _ in range(K)]
+    sampler = ClockSampler(None)
+    sampler.start()
+    for i in range(K):
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    call_ms = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
+    admit_ms = sum(call_ms)
+    total_bytes = K * sum(launch_bytes)
+    achieved = total_bytes / (admit_ms / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    traffic_per_group = profiled_traffic(ADMIT_PROFILE, ADMIT_SOURCES, "traffic_bytes_per_group_admit")
+    line = {
+        "metric": f"RMA admit GB/s (algorithmic), batch {B} x {L} layers, every bank and pending buffer full",
+        "value": achieved, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": admit_ms / K, "higher_is_better": True, "dtype": "u64", "data": "synthetic",
+        "config": {"workload": f"admit: {B} sequences x {L} RMA layers x {G} KV groups, all in phase (banks full "
+                               "with 1024 anchors, pending full with 256 candidates, scores ~ N(0,1)); one step = "
+                               "rma_admit per layer",
+                   "batch": B, "layers": L, "groups_per_launch": B * G,
+                   "admitted_per_group_mean": float(n_adm.mean()),
+                   "admitted_counts_match_kernel": counts_agree,
+                   "l2": "inputs larger than L2: each launch reads its layer's pending K/V "
+                         f"({B * G * 256 * 1024 / 1e9:.2f} GB) and writes into its bank "
+                         f"({B * G * 1024 * 1024 / 1e9:.2f} GB); the {score0.numel() * 4 / 1e6:.0f} MB of bank "
+                         "scores restored before each step (untimed) may sit in L2"},
+        "clocks": clocks,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic_per_group * B * G if traffic_per_group is not None else None,
+                     "traffic_note": "DRAM bytes per group from profiles/rma_admit_batch512.md (a 512-group "
+                                     "capture) x the groups of one launch",
+                     "kernel": "rma_admit (admit_kernel)", "kernel_ms": admit_ms,
+                     "algorithmic_bytes_per_launch": sum(launch_bytes) / L,
+                     "algorithmic_bytes_note": "5,120 B of scores per group + 2,052 B per admitted candidate "
+                                               "(K and V rows read and written, its score written)",
+                     "call_ms_mean": admit_ms / len(call_ms),
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s"},
+        "gpu_launches": K * L,
+    }
+    if not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = cpu_oracle_admit()
+        except Exception as ex:   # a report, never a reason to lose the bench line
+            line["cpu_baseline"] = {"value": None, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "sample": f"failed: {ex}"}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # the CUDA arm
 # ---------------------------------------------------------------------------
@@ -473,8 +618,9 @@ def main():
     ap.add_argument("--steps", type=int, default=1024)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--workload", default="batch", choices=["batch", "long", "ragged", "prefill"])
+    ap.add_argument("--workload", default="batch", choices=["batch", "long", "ragged", "prefill", "admit"])
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--layers", type=int, default=None, help="admit workload: RMA layers (default 8)")
     ap.add_argument("--blocks", type=int, default=128, help="prefill workload: blocks of 256 tokens")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -486,6 +632,11 @@ def main():
         return
     if args.workload == "prefill":
         run_prefill(args)
+        return
+    if args.workload == "admit":
+        if args.steps == 1024:       # the decode default; the admit workload takes fewer steps
+            args.steps = 20
+        run_admit(args)
         return
 
     import torch

@@ -48,3 +48,20 @@ def test_fill_tracker_full_state_is_the_published_per_step_figure():
     cnt[..., 1] = 1024
     tr = bench.FillTracker(cnt)
     assert tr.launch_bytes(0) == 512 * bench.BYTES_FULL == 512 * 8_409_088
+
+
+def test_admitted_counts_match_the_oracle_admit():
+    """`bench.admitted_counts` (the admit workload's byte count) against the oracle's own admit on
+    groups with every slot filled and 16-level scores (many ties, so the tie-break decides): the
+    bank rows the admit replaced are the admitted candidates."""
+    R, A, P, L, B, G = 5, 40, 12, 1, 6, 4
+    cfg = oracle.Config(batch=B, n_layers=L, ring_slots=R, bank_slots=A, pend_slots=P)
+    cont = si.state_contents(L, B, G, 256, R, A, P, seed=11, quantized_scores=True)
+    st = oracle.state_from_arrays(cfg, {k: to_np(v) for k, v in cont.items()}, pos=100, bank_fill=A, pend_fill=P)
+    counts = bench.admitted_counts(st.bank_score.copy(), st.pend_score.copy())
+    before = st.bank_k.copy()
+    oracle.admit(st, 0)
+    replaced = (st.bank_k != before).any(axis=-1).sum(axis=-1)
+    assert counts.shape == (L, B, G)
+    assert np.array_equal(counts, replaced)
+    assert 0 < counts.min() and counts.max() < P
