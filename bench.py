@@ -570,7 +570,8 @@ def run_admit(args) -> None:
     total_bytes = K * sum(launch_bytes)
     achieved = total_bytes / (admit_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
-    traffic_per_group = profiled_traffic(ADMIT_PROFILE, ADMIT_SOURCES, "traffic_bytes_per_group_admit")
+    # DRAM bytes of one full-size launch (2,048 groups), captured on this workload's default shape
+    traffic = profiled_traffic(ADMIT_PROFILE, ADMIT_SOURCES, "traffic_bytes_per_launch_admit") if B == 512 else None
     line = {
         "metric": f"RMA admit GB/s (algorithmic), batch {B} x {L} layers, every bank and pending buffer full",
         "value": achieved, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
@@ -587,9 +588,9 @@ def run_admit(args) -> None:
                          "scores restored before each step (untimed) may sit in L2"},
         "clocks": clocks,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic_per_group * B * G if traffic_per_group is not None else None,
-                     "traffic_note": "DRAM bytes per group from profiles/rma_admit_batch512.md (a 512-group "
-                                     "capture) x the groups of one launch",
+                     "traffic": traffic,
+                     "traffic_note": "DRAM read + write of one launch of 2,048 groups (layer 0, first timed "
+                                     "step), profiles/rma_admit_batch512.md",
                      "kernel": "rma_admit (admit_kernel)", "kernel_ms": admit_ms,
                      "algorithmic_bytes_per_launch": sum(launch_bytes) / L,
                      "algorithmic_bytes_note": "5,120 B of scores per group + 2,052 B per admitted candidate "

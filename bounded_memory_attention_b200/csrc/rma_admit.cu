@@ -21,8 +21,8 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// One CTA per (b, g).
-__global__ void __launch_bounds__(kThreads) admit_kernel(const __grid_constant__ LayerView s, int force) {
+// One CTA per (b, g); four CTAs per SM (64 registers a thread) keep more groups in flight.
+__global__ void __launch_bounds__(kThreads, 4) admit_kernel(const __grid_constant__ LayerView s, int force) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int g = blockIdx.x, b = blockIdx.y;
     const int bg = b * s.G + g;
