@@ -43,6 +43,9 @@ repository's design notes):
   * a decode step that finds the pending buffer full drops its candidate and
     raises STATUS_PENDING_OVERFLOW; a prefill block whose candidates do not fit
     drops them and raises STATUS_PREFILL_PENDING_OVERFLOW;
+  * a prefill block may hold any number n of tokens (the last block of a prompt
+    whose length is not a multiple of 256 is shorter); it appends after the
+    candidates still pending and always ends with the forced admit;
   * Q and K arrive already position-encoded (no RoPE inside the layer).
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
