@@ -43,12 +43,9 @@ __global__ void __launch_bounds__(kThreads, 4) admit_kernel(const __grid_constan
 
 cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream) {
     const size_t smem = admit_scratch_bytes(s.A, s.P);
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(admit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = smem;
-    }
+    static SmemLimit limit(reinterpret_cast<const void*>(admit_kernel));
+    const cudaError_t e = limit.ensure(smem);
+    if (e != cudaSuccess) return e;
     dim3 grid(s.G, s.B);
     admit_kernel<<<grid, kThreads, smem, stream>>>(s, force);
     return cudaGetLastError();

@@ -488,12 +488,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static SmemLimit limit(reinterpret_cast<const void*>(decode_kernel));
+    const cudaError_t e = limit.ensure(kSmemBytes);
+    if (e != cudaSuccess) return e;
     if (a.ring_splits + a.bank_splits > kMaxSplits) return cudaErrorInvalidValue;
     dim3 grid(a.ring_splits + a.bank_splits, a.s.G, a.s.B);
     decode_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);

@@ -4,9 +4,43 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
 #include "rma.h"
 
 namespace rma {
+
+// A kernel's dynamic shared-memory limit, raised past the default 48 KiB the first time a
+// launch on a device needs more.  The attribute belongs to the kernel as loaded on each
+// device, so the largest size set is tracked per device (devices past the first 64 set it
+// on every launch).  Safe to call from several host threads.
+class SmemLimit {
+  public:
+    explicit SmemLimit(const void* func) : func_(func) {}
+
+    cudaError_t ensure(size_t bytes) {
+        if (bytes <= 48 * 1024) return cudaSuccess;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const bool tracked = dev >= 0 && dev < kTracked;
+        if (tracked && set_[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        // never lower a limit another thread raised for a larger launch on this device
+        const size_t want = tracked ? std::max(bytes, set_[dev].load(std::memory_order_relaxed)) : bytes;
+        e = cudaFuncSetAttribute(func_, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)want);
+        if (e == cudaSuccess && tracked) set_[dev].store(want, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    static constexpr int kTracked = 64;
+    const void* func_;
+    std::mutex mu_;
+    std::atomic<size_t> set_[kTracked] = {};
+};
 
 constexpr int kHeadDim = 256;        // D: elements per K/V/Q row
 constexpr int kQPerGroup = 4;        // H: query heads reading one KV group

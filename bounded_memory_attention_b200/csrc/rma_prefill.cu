@@ -759,12 +759,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
               make_map(&tm.bank_k, s.bank_k, s.A, (uint64_t)B * G, row, row * s.A, kHalfKeys, 1) &&
               make_map(&tm.bank_v, s.bank_v, s.A, (uint64_t)B * G, row, row * s.A, kChunk, 1);
     if (!ok) return cudaErrorInvalidValue;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static SmemLimit limit(reinterpret_cast<const void*>(prefill_kernel));
+    const cudaError_t e = limit.ensure(kSmemBytes);
+    if (e != cudaSuccess) return e;
     // grid x: clusters of 4 CTAs, one per pair of tiles; ranks (local, local, anchor, anchor)
     prefill_kernel<<<dim3(2 * ntiles, G, B), kThreads, kSmemBytes, stream>>>(tm, a, ntiles);
     return cudaGetLastError();
