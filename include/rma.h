@@ -73,7 +73,10 @@ extern "C" {
 #define RMA_STATUS_BAD_COUNTERS              8u
 /* A kernel gave up waiting on one of its own pipeline barriers (a bounded
  * wait of about two seconds ran out) and abandoned its tile; its outputs are
- * not valid.  Indicates a fault in the library, never an input condition. */
+ * not valid, and the state of the groups it served (slots, counters,
+ * tickets) may be inconsistent: restore the state buffer from a copy or lay
+ * it out afresh with rma_state_alloc before the next call on it.  Indicates
+ * a fault in the library, never an input condition. */
 #define RMA_STATUS_TIMEOUT                  16u
 
 /* Dimensions.  The library implements q_per_group == 4 and head_dim == 256
