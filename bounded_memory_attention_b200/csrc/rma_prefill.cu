@@ -575,6 +575,12 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------- tail ----------------
     // The local CTA of this tile combines rows [0, 64), the anchor CTA rows [64, 128): each first
     // pushes the 64 rows the other one needs into that CTA's free stage area [128 KiB, 192 KiB).
+    // After a bounded wait ran out (this CTA abandoned its tile), the copies and tensor-core operations
+    // it had already issued are given ~2 ms to land before the stage area is reused and the CTA exits.
+    if (*abort_flag) {
+        for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+    }
+    __syncwarp();
     ptx::tc_fence_before();
     ptx::cluster_sync();   // all four CTAs have their rows in shared memory; all tensor memory reads done
     if (has_work && warp == kWarpQK) {
