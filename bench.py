@@ -47,10 +47,7 @@ UNIT = "tokens/s"
 # ring K+V 4*1023*1024, bank K+V 4*1024*1024, q 8192, out 8192, k_cur+v_cur 4096, ring write 4096
 BYTES_FULL = 4 * 1023 * 1024 + 4 * 1024 * 1024 + 8192 + 8192 + 4096 + 4096
 FALLBACK_HBM_GBS = 6650.0
-DECODE_PROFILE = os.path.join(ROOT, "profiles", "rma_decode_batch512.md")
-PREFILL_PROFILE = os.path.join(ROOT, "profiles", "rma_prefill_block.md")
-ADMIT_PROFILE = os.path.join(ROOT, "profiles", "rma_admit_batch512.md")
-ADMIT_SOURCES = ("rma_admit.cu", "rma_admit_impl.cuh")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")   # DRAM bytes per launch from ncu captures
 # algorithmic bytes of one group's admit: the 1,024 + 256 scores read once, then for every
 # admitted candidate its K and V rows (1 KiB together) read from pending and written to the
 # bank, and its score written (the two counters written are left out)
@@ -81,27 +78,19 @@ def kernel_source_hash(name) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(profile_path: str, source: str, key: str = "traffic_bytes_per_launch_batch512"):
-    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source.
-
-    The summary holds a line '<key>: <int>' and a line
-    'kernel_source_sha256_16: <hash>'; a different hash means the kernel
-    changed since the counters were taken, and traffic is reported as null.
-    """
-    if not os.path.exists(profile_path):
-        return None
-    vals = {}
-    with open(profile_path) as f:
-        for line in f:
-            if ":" in line:
-                k, v = line.split(":", 1)
-                vals[k.strip().strip("`-* ")] = v.strip().strip("`* ")
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash(source):
-        return None
-    try:
-        return int(vals[key])
-    except (KeyError, ValueError):
-        return None
+def profiled_traffic(kernel: str):
+    """(DRAM bytes per launch, workload it was captured on) for `kernel` ("rma_decode",
+    "rma_prefill" or "rma_admit") from profiles/traffic.json, or (None, reason) when there is no
+    capture or the kernel's sources changed since it was taken (their hash differs)."""
+    if not os.path.exists(TRAFFIC_JSON):
+        return None, "no ncu capture"
+    with open(TRAFFIC_JSON) as f:
+        entry = json.load(f).get(kernel)
+    if not entry:
+        return None, "no ncu capture"
+    if entry.get("kernel_source_sha256_16") != kernel_source_hash(tuple(entry["sources"])):
+        return None, "kernel changed since the last ncu capture"
+    return int(entry["traffic_bytes_per_launch"]), entry["workload"]
 
 
 class FillTracker:
@@ -279,6 +268,110 @@ def cpu_oracle_decode(n_seq: int, n_layers: int, n_steps: int, seed: int = 0) ->
                       f"(decode + admit), FP64 numpy oracle, 1 thread; {dt:.1f} s", "cpu": host_cpu()}
 
 
+def _usable_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_decode_worker(seq: int, n_layers: int, n_steps: int, start, results) -> None:
+    """One process of the all-core baseline: one sequence of the batch-512 workload through
+    n_steps decode steps of n_layers layers (decode + admit), one thread; reports its seconds."""
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(batch=1, n_layers=n_layers)
+    cont = si.state_contents(n_layers, 1, 4, 256, 1023, 1024, 256, seed=seq)
+    c = si.workload_counters("batch", n_layers, 1, 4)
+    c["pos"] += seq % 256
+    c["pend_fill"] += seq % 256
+    st = oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, **c)
+    w, b = si.gate_params(n_layers, 16, 256, seq)
+    w, b = w.numpy(), b.numpy()
+    ins = [[{k: _np(v) for k, v in si.decode_inputs(1, 4, 4, 256, seed=1000 * s + l + 7 * seq).items()}
+            for l in range(n_layers)] for s in range(n_steps)]
+    start.wait()
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for s in range(n_steps):
+            for l in range(n_layers):
+                x = ins[s][l]
+                oracle.decode_step(st, l, x["q"], x["k_cur"], x["v_cur"], x["cand_k"], x["cand_v"],
+                                   x["cand_score"], w[l], b[l])
+                oracle.admit(st, l)
+        results.put(time.perf_counter() - t0)
+
+
+def _oracle_prefill_worker(seq: int, n_blocks: int, start, results) -> None:
+    """One process of the all-core prefill baseline: steady-state blocks of one sequence and layer."""
+    import oracle
+    import synth_inputs as si
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(batch=1, n_layers=1)
+    cont = si.state_contents(1, 1, 4, 256, 1023, 1024, 256, seed=seq)
+    st = oracle.state_from_arrays(cfg, {k: _np(v) for k, v in cont.items()}, pos=4096, bank_fill=1024, pend_fill=0)
+    w, b = si.gate_params(1, 16, 256, seq)
+    xs = [{k: _np(v) for k, v in si.prefill_inputs(1, 256, 4, 4, 256, seed=100 * seq + j).items()}
+          for j in range(n_blocks)]
+    start.wait()
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        for x in xs:
+            oracle.prefill_block(st, 0, x["q"], x["k"], x["v"], x["cand_k"], x["cand_v"], x["cand_score"],
+                                 w[0].numpy(), b[0].numpy())
+        results.put(time.perf_counter() - t0)
+
+
+def _all_cores(target, args_of, n_proc: int) -> float:
+    """Run target(*args_of(i), start, results) in n_proc spawned processes (spawn: the parent may
+    hold a CUDA context), release them together once all are set up, and return the seconds
+    from the release until the last one finishes its timed work."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    start, results = ctx.Event(), ctx.Queue()
+    procs = [ctx.Process(target=target, args=(*args_of(i), start, results)) for i in range(n_proc)]
+    for p in procs:
+        p.start()
+    time.sleep(0.5)
+    # wait until every worker has built its inputs (they block on `start` with little CPU use)
+    deadline = time.time() + 300
+    while time.time() < deadline and any(p.is_alive() for p in procs):
+        import psutil
+        busy = sum(psutil.Process(p.pid).cpu_percent(interval=0.2) > 20 for p in procs if p.is_alive())
+        if busy == 0:
+            break
+    t0 = time.perf_counter()
+    start.set()
+    for _ in procs:
+        results.get(timeout=600)
+    dt = time.perf_counter() - t0
+    for p in procs:
+        p.join(timeout=60)
+    return dt
+
+
+def cpu_oracle_decode_allcores(n_steps: int = 2, n_layers: int = 8) -> dict:
+    """The oracle on every usable host core: one process per core, each one sequence of the
+    batch-512 workload through n_steps steps of n_layers layers; tokens/s over all of them."""
+    n = _usable_cores()
+    dt = _all_cores(_oracle_decode_worker, lambda i: (i, n_layers, n_steps), n)
+    return {"value": n * n_steps / dt, "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{n} of the 512 sequences (one process per core) x {n_layers} layers x {n_steps} steps "
+                      f"(decode + admit), FP64 numpy oracle; {dt:.1f} s", "cpu": host_cpu()}
+
+
+def cpu_oracle_prefill_allcores(n_blocks: int = 2) -> dict:
+    """The oracle on every usable host core: one process per core, each steady-state blocks of
+    its own sequence at one layer; algorithmic GFLOP/s over all of them."""
+    n = _usable_cores()
+    dt = _all_cores(_oracle_prefill_worker, lambda i: (i, n_blocks), n)
+    flops = prefill_flops(1, 1, 256, 20)[-1] * n_blocks * n
+    return {"value": flops / dt / 1e9, "unit": "GFLOP/s", "cores": n, "kind": "oracle",
+            "sample": f"{n} sequences (one process per core) x {n_blocks} blocks of 256 tokens at one layer (ring and "
+                      f"bank full, forced admits), FP64 numpy oracle; {dt:.1f} s", "cpu": host_cpu()}
+
+
 def host_cpu() -> str:
     """The host CPU's model name and logical core count."""
     model = "unknown CPU"
@@ -446,6 +539,7 @@ def run_prefill(args) -> None:
         pk = json.load(f)
     peak = float(pk["bf16_tflops_sustained"])
     achieved = total_flops / (sum(call_ms) / 1e3) / 1e12
+    pf_traffic, pf_traffic_note = profiled_traffic("rma_prefill")
     line = {
         "metric": f"RMA block-prefill TFLOP/s (algorithmic), batch {B} x {L} layers x {blocks} blocks of {n}",
         "value": total_flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "tokens_per_s": B * n * blocks / (ms / 1e3),
@@ -460,8 +554,7 @@ def run_prefill(args) -> None:
         "clocks": clocks,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "traffic": profiled_traffic(PREFILL_PROFILE, "rma_prefill.cu", "traffic_bytes_per_launch_prefill"),
-                     "traffic_note": "one steady-state launch (ring and bank full), profiles/rma_prefill_block.md",
+                     "traffic": pf_traffic, "traffic_note": pf_traffic_note,
                      "kernel": "rma_prefill_block (one launch: attention, commit, forced admit)",
                      "call_ms_mean": sum(call_ms) / len(call_ms),
                      "peak_source": "measured bf16_tflops_sustained (MEASURED_PEAKS.json)"},
@@ -571,7 +664,7 @@ def run_admit(args) -> None:
     achieved = total_bytes / (admit_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
     # DRAM bytes of one full-size launch (2,048 groups), captured on this workload's default shape
-    traffic = profiled_traffic(ADMIT_PROFILE, ADMIT_SOURCES, "traffic_bytes_per_launch_admit") if B == 512 else None
+    traffic, traffic_note = profiled_traffic("rma_admit") if B == 512 else (None, "captured at batch 512 only")
     line = {
         "metric": f"RMA admit GB/s (algorithmic), batch {B} x {L} layers, every bank and pending buffer full",
         "value": achieved, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
@@ -588,9 +681,7 @@ def run_admit(args) -> None:
                          "scores restored before each step (untimed) may sit in L2"},
         "clocks": clocks,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic,
-                     "traffic_note": "DRAM read + write of one launch of 2,048 groups (layer 0, first timed "
-                                     "step), profiles/rma_admit_batch512.md",
+                     "traffic": traffic, "traffic_note": traffic_note,
                      "kernel": "rma_admit (admit_kernel)", "kernel_ms": admit_ms,
                      "algorithmic_bytes_per_launch": sum(launch_bytes) / L,
                      "algorithmic_bytes_note": "5,120 B of scores per group + 2,052 B per admitted candidate "
@@ -752,6 +843,8 @@ def main():
         durs = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
         dec_ms = sum(durs) / len(durs)
     alg_bytes = sum(timed_bytes) / (K * L)     # per launch, from the exact per-step fills
+    dec_traffic, dec_traffic_note = (profiled_traffic("rma_decode") if kind == "batch"
+                                     else (None, "captured on the batch-512 workload only"))
     peak, peak_kind = peaks()
 
     # end to end through the public API: host (pinned) inputs in, host output out, every step
@@ -850,7 +943,7 @@ def main():
                          "achieved": (alg_bytes / (dec_ms / 1e3) / 1e9) if alg_bytes else None,
                          "peak": peak, "unit": "GB/s",
                          "frac": (alg_bytes / (dec_ms / 1e3) / 1e9 / peak) if alg_bytes else None,
-                         "traffic": profiled_traffic(DECODE_PROFILE, "rma_decode.cu") if kind == "batch" else None,
+                         "traffic": dec_traffic, "traffic_note": dec_traffic_note,
                          "kernel": "rma_decode (decode_kernel)", "kernel_ms": dec_ms,
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "algorithmic_bytes_note": "ring min(pos, 1023) + bank_fill rows x 1 KiB per group, plus "

@@ -144,15 +144,24 @@ class State:
     listed in include/rma.h (counters [L, B, G, 4] = pos, bank_fill, pend_fill, 0).
     """
 
-    def __init__(self, cfg: Config, device=None, stream=None):
+    def __init__(self, cfg: Config, device=None, stream=None, buffer: torch.Tensor = None):
+        """Lay a state out over `buffer` (a CUDA uint8 tensor, 256-byte aligned, at least
+        state_bytes(cfg) bytes, e.g. a view into a larger allocation), or over a fresh one."""
         self.cfg = cfg
         n = state_bytes(cfg)
         if n == 0:
             raise ValueError(f"invalid RMA config: {lib.rma_last_error().decode()}")
-        device = torch.device(device if device is not None else "cuda")
-        self.buffer = torch.empty(n + 256, dtype=torch.uint8, device=device)
-        off = (-self.buffer.data_ptr()) % 256
-        self.buffer = self.buffer[off:off + n]
+        if buffer is not None:
+            if buffer.dtype != torch.uint8 or not buffer.is_cuda or not buffer.is_contiguous():
+                raise TypeError("buffer must be a contiguous CUDA uint8 tensor")
+            if buffer.numel() < n:
+                raise ValueError(f"buffer holds {buffer.numel()} bytes, the state needs {n}")
+            self.buffer = buffer[:n]
+        else:
+            device = torch.device(device if device is not None else "cuda")
+            self.buffer = torch.empty(n + 256, dtype=torch.uint8, device=device)
+            off = (-self.buffer.data_ptr()) % 256
+            self.buffer = self.buffer[off:off + n]
         self._h = ctypes.c_void_p()
         c = cfg._c()
         _check(lib.rma_state_alloc(ctypes.byref(c), ctypes.c_void_p(self.buffer.data_ptr()), n,

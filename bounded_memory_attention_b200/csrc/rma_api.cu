@@ -5,6 +5,8 @@
 #include <new>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "rma_internal.cuh"
 
 namespace rma {
@@ -20,6 +22,15 @@ int fail(int code, const std::string& why) {
 int cuda_fail(cudaError_t e, const char* what) {
     return fail(RMA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
+
+// An NVTX range named after the API call around its host work and launches, so that a
+// profiler's launch list shows which call issued each kernel (no cost without a profiler).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr uint64_t kAlign = 256;
 constexpr int kMaxDecodeSplits = 64;   // must match the decode kernel's kMaxSplits
@@ -96,12 +107,13 @@ struct Splits {
     int ring_splits, bank_splits, ring_chunk, bank_chunk;
 };
 
-// Cut `rows` into at most `want` contiguous ranges of a multiple of 4 rows.
+// Cut `rows` into at most `want` contiguous ranges of a multiple of 16 rows (the decode
+// kernel's tensor-core tile).
 void cut(int rows, int want, int& n, int& chunk) {
     want = want < 1 ? 1 : want;
     chunk = (rows + want - 1) / want;
-    chunk = (chunk + 3) / 4 * 4;
-    if (chunk < 4) chunk = 4;
+    chunk = (chunk + 15) / 16 * 16;
+    if (chunk < 16) chunk = 16;
     n = (rows + chunk - 1) / chunk;
 }
 
@@ -109,13 +121,14 @@ Splits decode_splits(const State& s) {
     const rma_config& c = s.cfg;
     int want_r = s.ring_splits_override, want_b = s.bank_splits_override;
     if (want_r <= 0 || want_b <= 0) {
-        // enough CTAs to fill every SM several times over, without cutting
-        // rows so thin that the per-split merge dominates
+        // one CTA per SM at a time: about four waves of CTAs, without cutting rows so
+        // thin that the per-split merge dominates (at most 8 + 8 splits, 128 rows each
+        // for the pages' ring and bank)
         const long units = (long)c.batch * c.n_groups;
-        const long target = (long)s.sm_count * 8;
+        const long target = (long)s.sm_count * 4;
         long per_unit = (target + units - 1) / units;
         if (per_unit < 2) per_unit = 2;
-        if (per_unit > 32) per_unit = 32;
+        if (per_unit > 16) per_unit = 16;
         want_r = (int)(per_unit / 2);
         want_b = (int)(per_unit - per_unit / 2);
     }
@@ -218,6 +231,7 @@ int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_splits) {
 int rma_decode_step(rma_state* st, int layer, const uint16_t* q, const uint16_t* k_cur, const uint16_t* v_cur,
                     const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score, const float* w_g,
                     const float* b_g, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange range("rma_decode_step");
     State* s = as_state(st);
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;
@@ -257,6 +271,7 @@ int rma_decode_step_noalloc(rma_state* st, int layer, const uint16_t* q, const u
                             const uint16_t* v_cur, const uint16_t* cand_k, const uint16_t* cand_v,
                             const float* cand_score, const float* w_g, const float* b_g, uint16_t* out,
                             void* stream) {
+    NvtxRange range("rma_decode_step_noalloc");
     State* s = as_state(st);
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;
@@ -277,6 +292,7 @@ int rma_decode_step_noalloc(rma_state* st, int layer, const uint16_t* q, const u
 }
 
 int rma_admit(rma_state* st, int layer, int force, void* stream) {
+    NvtxRange range("rma_admit");
     State* s = as_state(st);
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;
@@ -289,6 +305,7 @@ int rma_admit(rma_state* st, int layer, int force, void* stream) {
 int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                       const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score, const float* w_g,
                       const float* b_g, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange range("rma_prefill_block");
     State* s = as_state(st);
     int rc = check_layer(s, layer);
     if (rc != RMA_OK) return rc;

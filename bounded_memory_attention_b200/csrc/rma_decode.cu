@@ -9,44 +9,55 @@
 // then writes the current K/V into ring slot pos mod R and appends the
 // candidate record to the pending buffer.
 //
-// Design (HBM-bound; ~2 FMA per byte streamed):
+// Design (HBM-bound: every K/V byte is read once, ~2 FLOP per byte):
 //   grid = (ring_splits + bank_splits, G, B).  Each CTA streams one contiguous
-//   row range of one (b, g)'s ring or bank.  Rows are processed in tiles of 4;
-//   warp w takes tiles w, w + W, w + 2W, ... and runs its OWN cp.async
-//   pipeline (each lane copies, and later reads, exactly its own 16-byte
-//   column of each row, so no block barrier is needed while streaming).
-//   A lane holds 8 of the 256 dims for all 4 heads: QK^T is 32 FMAs per row
-//   per lane, reduced across lanes by a 16-value reduce-scatter (16 shuffles
-//   per 4 rows); the online softmax (log2 domain) and P.V run in FP32 with
-//   packed FFMA2.  Warps merge in shared memory into one (m, l, acc) partial
-//   per CTA; the last CTA of (b, g) to arrive (atomic ticket, no waiting)
-//   merges all partials, adds the current token and the gate, writes the
-//   output and performs the state writes after every read of the step; when
-//   the step fills the pending buffer it also runs the admit for (b, g).
+//   row range of one (b, g)'s ring or bank in tiles of 16 rows.  Warp w takes
+//   tiles w, w + 8, w + 16, ... with its own K slot and V slot in shared
+//   memory: the lanes copy a tile's rows with one 512-byte bulk copy each
+//   (completion counted on the slot's mbarrier) into rows padded to 528 bytes,
+//   so that the tensor-core fragment loads below are free of bank conflicts.
+//   The next tile's K is requested as soon as this tile's Q K^T has read its
+//   K slot, its V as soon as P V has read the V slot.
+//   Both products run on the tensor cores (mma.sync m16n8k16, BF16 operands,
+//   FP32 accumulation), with the 16 keys of the tile in M and the group's
+//   heads in N (4 of the 8 columns used):
+//     S^T [16 keys x 8]  = K [16 x 256] . Q^T [256 x 8]     (K from ldmatrix)
+//     O^T [256 x 8]     += V^T [256 x 16] . P^T [16 x 8]    (V from ldmatrix.trans)
+//   The softmax runs on S^T in registers (log2 domain, FP32; the running max
+//   moves, and O is rescaled, only when a tile raises it); P is rounded to
+//   BF16 and turned from the S^T accumulator layout into the P^T operand
+//   layout with movmatrix.  Warps merge in shared memory into one (m, l, acc)
+//   partial per CTA; the last CTA of (b, g) to arrive (atomic ticket, no
+//   waiting) merges all partials, adds the current token and the gate, writes
+//   the output and performs the state writes after every read of the step;
+//   when the step fills the pending buffer it also runs the admit for (b, g).
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
-#include <mutex>
-
 #include "rma_admit_impl.cuh"
 #include "rma_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace rma {
 namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 3;
-constexpr int kTileRows = 4;
-constexpr int kStageBytes = 2 * kTileRows * kRowBytes;          // K tile + V tile = 4 KiB
-constexpr int kPipeBytes = kWarps * kStages * kStageBytes;       // 96 KiB
-constexpr int kBcastFloats = 32;                                 // per warp: 16 p + 4 alpha (+pad)
+constexpr int kTile = 16;                                        // keys per tensor-core tile
+constexpr int kRowStride = kRowBytes + 16;                       // 528: padded shared-memory row
+constexpr int kSlotBytes = kTile * kRowStride;                   // 8,448: one K or V tile
+constexpr int kWarpRegion = 2 * kSlotBytes;                      // this warp's K slot + V slot
+constexpr int kPipeBytes = kWarps * kWarpRegion;                 // 135,168
 constexpr int kMaxSplits = 64;                                   // ring_splits + bank_splits
-constexpr int kSmemBytes = kPipeBytes + kWarps * kBcastFloats * 4 + (kMaxSplits + 1) * 4 * 4 + 16 * 4;
+constexpr int kCoefOff = kPipeBytes;                             // [(kMaxSplits + 1)][4] floats
+constexpr int kMiscOff = kCoefOff + (kMaxSplits + 1) * 4 * 4;    // scur[4], gate[4] (+ pad)
+constexpr int kBarOff = kMiscOff + 16 * 4;                       // [kWarps][2] mbarriers
+constexpr int kSmemBytes = kBarOff + kWarps * 2 * 8;
 
 static_assert(kWarps == 8, "merger assigns 8 dot products to 8 warps");
-static_assert(kStages * kStageBytes >= kPartialFloats * 4, "per-warp pipeline region must hold one warp partial");
-static_assert(kPipeBytes >= admit_scratch_bytes(1, 4095), "the admit reuses the pipeline region (any A + P <= 4096)");
+static_assert(kSlotBytes >= kPartialFloats * 4, "a warp's K slot must hold one warp partial");
+static_assert(kPipeBytes >= (int)admit_scratch_bytes(1, 4095), "the admit reuses the pipeline region (any A + P <= 4096)");
+static_assert((kBarOff & 7) == 0, "mbarriers are 8-byte aligned");
 
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -58,22 +69,56 @@ __device__ __forceinline__ float fast_ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes));
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     uint4 r;
     asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
     return r;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.u32 %0, [%1];\n" : "=r"(r) : "l"(p));
+    return r;
+}
+
+// `bytes` (a multiple of 16) from global memory to this CTA's shared memory, counted as tx
+// bytes on the mbarrier `bar`; a plain copy into this CTA (no multicast).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Four 8x8 BF16 matrices from shared memory (lane L gives the address of row L & 7 of matrix L >> 3).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+// D (16x8 FP32) += A (16x16 BF16, row) . B (16x8 BF16, col)
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit values held one row pair per lane in the mma fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -96,52 +141,31 @@ __device__ __forceinline__ float dot8(const float2 (&q)[4], const uint4& k) {
     return d.x + d.y;
 }
 
-// Reduce 16 per-lane partial sums across the warp so that lane L ends up
-// with the full sum of value index (L >> 1) & 15 (lanes L and L^1 agree).
-__device__ __forceinline__ float reduce_scatter16(float (&x)[16], int lane) {
-    {
-        const bool up = lane & 16;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float send = up ? x[i] : x[i + 8];
-            float keep = up ? x[i + 8] : x[i];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+// Bounded wait on an mbarrier phase (about two seconds); on timeout sets RMA_STATUS_TIMEOUT and
+// returns false.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > ptx::kWaitLimitCycles) {
+            atomicOr(status, (unsigned)RMA_STATUS_TIMEOUT);
+            return false;
         }
     }
-    {
-        const bool up = lane & 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            float send = up ? x[i] : x[i + 4];
-            float keep = up ? x[i + 4] : x[i];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-    }
-    {
-        const bool up = lane & 4;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            float send = up ? x[i] : x[i + 2];
-            float keep = up ? x[i + 2] : x[i];
-            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        }
-    }
-    {
-        const bool up = lane & 2;
-        float send = up ? x[0] : x[1];
-        float keep = up ? x[1] : x[0];
-        x[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-    return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+    return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.s.G;
     const int bg = b * G + g;
     const int n_splits = a.ring_splits + a.bank_splits;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+    if (tid < 2 * kWarps) ptx::mbar_init(&bars[tid], 1);
+    ptx::fence_mbar_init();
 
     const int32_t* cnt = a.s.counters + bg * 4;
     int pos = cnt[0], bank_fill = cnt[1], pend_fill = cnt[2];
@@ -172,129 +196,166 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         kbase = a.s.bank_k + off;
         vbase = a.s.bank_v + off;
     }
+    __syncthreads();   // the mbarriers are initialised
 
-    // ---- per-warp cp.async pipeline over this warp's tiles ----
-    uint8_t* wsm = smem + warp * (kStages * kStageBytes);
-    const uint32_t wsm_a = smem_addr(wsm);
-    float* bc = reinterpret_cast<float*>(smem + kPipeBytes) + warp * kBcastFloats;
-    const int n_tiles = (nrows + kTileRows - 1) / kTileRows;
+    // ---- this warp's tiles: w, w + 8, ...; K slot and V slot, one mbarrier each ----
+    uint8_t* wsm = smem + warp * kWarpRegion;
+    const uint32_t kslot = ptx::smem_u32(wsm), vslot = kslot + kSlotBytes;
+    uint64_t* kbar = &bars[2 * warp];
+    uint64_t* vbar = &bars[2 * warp + 1];
+    const int n_tiles = (nrows + kTile - 1) / kTile;
     const int my_n = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
 
-    auto issue = [&](int i, int stage) {
-        const int t = warp + i * kWarps;
-        const uint32_t dst = wsm_a + stage * kStageBytes + lane * 16;
-#pragma unroll
-        for (int j = 0; j < kTileRows; ++j) {
-            const int r = t * kTileRows + j;
-            const bool ok = r < nrows;
-            const size_t roff = (size_t)(ok ? r : 0) * kHeadDim + lane * 8;
-            cp_async16(dst + j * kRowBytes, kbase + roff, ok ? 16 : 0);
-            cp_async16(dst + (kTileRows + j) * kRowBytes, vbase + roff, ok ? 16 : 0);
-        }
+    // rows of tile i of this warp -> one slot: lane r < rows copies row r (512 bytes)
+    auto issue = [&](int i, bool v_half) {
+        const int r0 = (warp + i * kWarps) * kTile;
+        const int nv = min(kTile, nrows - r0);
+        uint64_t* bar = v_half ? vbar : kbar;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(bar, (uint32_t)(nv * kRowBytes));
+        __syncwarp();
+        if (lane < nv)
+            bulk_g2s((v_half ? vslot : kslot) + lane * kRowStride, (v_half ? vbase : kbase) + (size_t)(r0 + lane) * kHeadDim,
+                     kRowBytes, ptx::smem_u32(bar));
     };
-
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-        if (s < my_n) issue(s, s);
-        cp_commit();
+    if (my_n > 0) {
+        issue(0, false);
+        issue(0, true);
     }
 
-    // ---- q of the group's 4 heads, this lane's 8 dims, in the log2 domain (loaded while the
-    //      first K/V tiles are in flight) ----
-    float2 q2[kQPerGroup][4];
+    // ---- Q^T fragments (the B operand of S^T = K Q^T), loaded while the first tiles are in flight:
+    //      lane (gq = lane / 4, tq = lane % 4) holds head gq's dims 16 c + 2 tq (+1) and 16 c + 2 tq + 8 (+9);
+    //      heads 4..7 of the 8 columns are zero ----
+    const int gq = lane >> 2, tq = lane & 3;
     const uint16_t* qg = a.q + ((size_t)b * G * kQPerGroup + (size_t)g * kQPerGroup) * kHeadDim;
+    uint32_t qf[16][2];
 #pragma unroll
-    for (int h = 0; h < kQPerGroup; ++h) {
-        const uint4 r = ld_nc_v4(qg + h * kHeadDim + lane * 8);
-        const float2 s2 = make_float2(a.qscale, a.qscale);
-        q2[h][0] = __fmul2_rn(bf2_to_f2(r.x), s2);
-        q2[h][1] = __fmul2_rn(bf2_to_f2(r.y), s2);
-        q2[h][2] = __fmul2_rn(bf2_to_f2(r.z), s2);
-        q2[h][3] = __fmul2_rn(bf2_to_f2(r.w), s2);
+    for (int c = 0; c < 16; ++c) {
+        qf[c][0] = gq < kQPerGroup ? ld_nc_u32(qg + gq * kHeadDim + 16 * c + 2 * tq) : 0u;
+        qf[c][1] = gq < kQPerGroup ? ld_nc_u32(qg + gq * kHeadDim + 16 * c + 2 * tq + 8) : 0u;
     }
 
+    // ldmatrix row addresses: lane L feeds row L & 7 of matrix L >> 3
+    const int lr = lane & 7, lm = lane >> 3;
+    // K (A operand, rows = keys): matrices (keys 0-7 | 8-15) x (dims +0-7 | +8-15)
+    const uint32_t k_addr = kslot + (uint32_t)((lr + 8 * (lm & 1)) * kRowStride + 16 * (lm >> 1));
+    // V^T (A operand via .trans, rows = dims): matrices (dims +0-7 | +8-15) x (keys 0-7 | 8-15)
+    const uint32_t v_addr = vslot + (uint32_t)((lr + 8 * (lm >> 1)) * kRowStride + 16 * (lm & 1));
 
-    float m_run = -CUDART_INF_F, l_run = 0.f;
-    float2 acc[kQPerGroup][4];
+    // running softmax of heads 2 tq and 2 tq + 1 (lanes with tq >= 2 carry the unused columns)
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    float acc[16][4];
 #pragma unroll
-    for (int h = 0; h < kQPerGroup; ++h)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
+    for (int mt = 0; mt < 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    const float qs = a.qscale;
+    bool ok = true;
+    int k_issued = my_n > 0 ? 1 : 0, v_issued = k_issued;
 
-    const int my_j = (lane >> 3) & 3;   // row of the tile this lane's reduced score belongs to
-    const int my_h = (lane >> 1) & 3;   // head of this lane's reduced score
-
-    for (int i = 0; i < my_n; ++i) {
-        cp_wait<kStages - 1>();
-        const int stage = i % kStages;
-        const uint8_t* ks = wsm + stage * kStageBytes + lane * 16;
-        const uint8_t* vs = ks + kTileRows * kRowBytes;
-
-        float x[16];
+    for (int i = 0; i < my_n && ok; ++i) {
+        const int r0 = (warp + i * kWarps) * kTile;
+        const int nv = min(kTile, nrows - r0);
+        // ---- S^T = K Q^T: 16 MMAs in four independent chains ----
+        if (!wait_phase(kbar, i & 1, a.s.status)) { ok = false; break; }
+        float s[4][4];
 #pragma unroll
-        for (int j = 0; j < kTileRows; ++j) {
-            const uint4 kr = *reinterpret_cast<const uint4*>(ks + j * kRowBytes);
+        for (int c = 0; c < 4; ++c) s[c][0] = s[c][1] = s[c][2] = s[c][3] = 0.f;
 #pragma unroll
-            for (int h = 0; h < kQPerGroup; ++h) x[j * 4 + h] = dot8(q2[h], kr);
+        for (int c = 0; c < 16; ++c) {
+            uint32_t af[4];
+            ldsm_x4(k_addr + 32 * c, af);
+            mma_16816(s[c & 3], af, qf[c][0], qf[c][1]);
         }
-        float sc = reduce_scatter16(x, lane);
-        const int row = (warp + i * kWarps) * kTileRows + my_j;
-        if (row >= nrows) sc = -CUDART_INF_F;
-
-        float mx = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run, mx);
-        const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-        const float alpha = fast_ex2(m_run - m_use);
-        const float p = fast_ex2(sc - m_use);
-        float ps = p + __shfl_xor_sync(0xffffffffu, p, 8);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-        l_run = l_run * alpha + ps;
-        m_run = m_new;
-
         __syncwarp();
-        if ((lane & 1) == 0) bc[(lane >> 1) & 15] = p;
-        if ((lane & 0x19) == 0) bc[16 + my_h] = alpha;
-        __syncwarp();
-        const float4 al = *reinterpret_cast<const float4*>(bc + 16);
-        const float alv[4] = {al.x, al.y, al.z, al.w};
-#pragma unroll
-        for (int h = 0; h < kQPerGroup; ++h) {
-            const float2 a2 = make_float2(alv[h], alv[h]);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[h][c] = __fmul2_rn(acc[h][c], a2);
+        if (i + 1 < my_n) {   // the K slot has been read: request the next tile's K
+            issue(i + 1, false);
+            ++k_issued;
         }
+        // ---- softmax on S^T: x0 = (key gq, head 2tq), x1 = (gq, 2tq+1), x2 = (gq+8, 2tq), x3 = (gq+8, 2tq+1) ----
+        const bool va = gq < nv, vb = gq + 8 < nv;
+        const float x0 = va ? ((s[0][0] + s[1][0]) + (s[2][0] + s[3][0])) * qs : -CUDART_INF_F;
+        const float x1 = va ? ((s[0][1] + s[1][1]) + (s[2][1] + s[3][1])) * qs : -CUDART_INF_F;
+        const float x2 = vb ? ((s[0][2] + s[1][2]) + (s[2][2] + s[3][2])) * qs : -CUDART_INF_F;
+        const float x3 = vb ? ((s[0][3] + s[1][3]) + (s[2][3] + s[3][3])) * qs : -CUDART_INF_F;
+        float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int j = 0; j < kTileRows; ++j) {
-            const float4 pj = *reinterpret_cast<const float4*>(bc + 4 * j);
-            const float pv[4] = {pj.x, pj.y, pj.z, pj.w};
-            const uint4 vr = *reinterpret_cast<const uint4*>(vs + j * kRowBytes);
-            const float2 v0 = bf2_to_f2(vr.x), v1 = bf2_to_f2(vr.y), v2 = bf2_to_f2(vr.z), v3 = bf2_to_f2(vr.w);
+        for (int o = 4; o < 32; o <<= 1) {
+            t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+            t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+        }
+        const bool up0 = t0 > m0, up1 = t1 > m1;
+        if (__any_sync(0xffffffffu, up0 || up1)) {
+            // the running max grew: rescale what this lane holds of those heads
+            const float f0 = up0 ? (m0 == -CUDART_INF_F ? 0.f : fast_ex2(m0 - t0)) : 1.f;
+            const float f1 = up1 ? (m1 == -CUDART_INF_F ? 0.f : fast_ex2(m1 - t1)) : 1.f;
+            m0 = up0 ? t0 : m0;
+            m1 = up1 ? t1 : m1;
+            l0 *= f0;
+            l1 *= f1;
 #pragma unroll
-            for (int h = 0; h < kQPerGroup; ++h) {
-                const float2 p2 = make_float2(pv[h], pv[h]);
-                acc[h][0] = __ffma2_rn(p2, v0, acc[h][0]);
-                acc[h][1] = __ffma2_rn(p2, v1, acc[h][1]);
-                acc[h][2] = __ffma2_rn(p2, v2, acc[h][2]);
-                acc[h][3] = __ffma2_rn(p2, v3, acc[h][3]);
+            for (int mt = 0; mt < 16; ++mt) {
+                acc[mt][0] *= f0;
+                acc[mt][1] *= f1;
+                acc[mt][2] *= f0;
+                acc[mt][3] *= f1;
             }
         }
-        if (i + kStages < my_n) issue(i + kStages, stage);
-        cp_commit();
-    }
-    cp_wait<0>();
-
-    // ---- merge the warps of this CTA (each warp's pipeline region holds its partial) ----
-    float* wpart = reinterpret_cast<float*>(wsm);
-    if ((lane & 0x19) == 0) {
-        wpart[my_h] = m_run;
-        wpart[4 + my_h] = l_run;
-    }
+        const float p0 = fast_ex2(x0 - m0), p1 = fast_ex2(x1 - m1);
+        const float p2 = fast_ex2(x2 - m0), p3 = fast_ex2(x3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        // P^T operand (k = key, n = head): transpose the two 8x8 BF16 blocks of P^T's rows
+        const uint32_t pb0 = movmatrix_trans(pack_bf16(p0, p1));
+        const uint32_t pb1 = movmatrix_trans(pack_bf16(p2, p3));
+        // ---- O^T += V^T P^T: 16 MMAs, one per 16 dims ----
+        if (!wait_phase(vbar, i & 1, a.s.status)) { ok = false; break; }
+        if (nv < kTile) {
+            // rows past the range hold stale bytes: zero them so that 0 x stale stays 0
+            for (int e = lane; e < (kTile - nv) * (kRowBytes / 16); e += 32)
+                *reinterpret_cast<uint4*>(wsm + kSlotBytes + (nv + e / (kRowBytes / 16)) * kRowStride +
+                                          16 * (e % (kRowBytes / 16))) = make_uint4(0, 0, 0, 0);
+            __syncwarp();
+        }
 #pragma unroll
-    for (int h = 0; h < kQPerGroup; ++h) {
-        float4* dst = reinterpret_cast<float4*>(wpart + 8 + h * kHeadDim + lane * 8);
-        dst[0] = make_float4(acc[h][0].x, acc[h][0].y, acc[h][1].x, acc[h][1].y);
-        dst[1] = make_float4(acc[h][2].x, acc[h][2].y, acc[h][3].x, acc[h][3].y);
+        for (int mt = 0; mt < 16; ++mt) {
+            uint32_t af[4];
+            ldsm_x4_trans(v_addr + 32 * mt, af);
+            mma_16816(acc[mt], af, pb0, pb1);
+        }
+        __syncwarp();
+        if (i + 1 < my_n) {   // the V slot has been read: request the next tile's V
+            issue(i + 1, true);
+            ++v_issued;
+        }
+    }
+    if (!ok) {
+        // a wait ran out: let the copies this warp already requested land before its slots are reused
+        if (k_issued > 0) wait_phase(kbar, (k_issued - 1) & 1, a.s.status);
+        if (v_issued > 0) wait_phase(vbar, (v_issued - 1) & 1, a.s.status);
+    }
+    // row sums over the 8 key rows of the fragment
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+
+    // ---- this warp's partial (m, l, acc) into its K slot: lanes with tq < 2 hold heads 0..3 ----
+    __syncwarp();
+    float* wpart = reinterpret_cast<float*>(wsm);
+    if (tq < 2) {
+        const int h0 = 2 * tq, h1 = 2 * tq + 1;
+        if (gq == 0) {
+            wpart[h0] = m0;
+            wpart[h1] = m1;
+            wpart[4 + h0] = l0;
+            wpart[4 + h1] = l1;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 16; ++mt) {
+            wpart[8 + h0 * kHeadDim + 16 * mt + gq] = acc[mt][0];
+            wpart[8 + h1 * kHeadDim + 16 * mt + gq] = acc[mt][1];
+            wpart[8 + h0 * kHeadDim + 16 * mt + gq + 8] = acc[mt][2];
+            wpart[8 + h1 * kHeadDim + 16 * mt + gq + 8] = acc[mt][3];
+        }
     }
     __syncthreads();
 
@@ -306,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         float M = -CUDART_INF_F;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            mw[w] = reinterpret_cast<const float*>(smem + w * (kStages * kStageBytes))[h];
+            mw[w] = reinterpret_cast<const float*>(smem + w * kWarpRegion)[h];
             M = fmaxf(M, mw[w]);
         }
         const float Mu = (M == -CUDART_INF_F) ? 0.f : M;
@@ -314,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
         float L = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float* wp = reinterpret_cast<const float*>(smem + w * (kStages * kStageBytes));
+            const float* wp = reinterpret_cast<const float*>(smem + w * kWarpRegion);
             const float c = fast_ex2(mw[w] - Mu);
             L += c * wp[4 + h];
             const float4 v = *reinterpret_cast<const float4*>(wp + 8 + h * kHeadDim + d);
@@ -339,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
     __threadfence();
 
     // ---- last CTA of (b, g): merge every split, add the current token, gate, write ----
-    float* coef = reinterpret_cast<float*>(smem + kPipeBytes + kWarps * kBcastFloats * 4);  // [(n_splits+1)][4]
-    float* misc = coef + (kMaxSplits + 1) * 4;                                             // scur[4], gate[4]
+    float* coef = reinterpret_cast<float*>(smem + kCoefOff);   // [(n_splits+1)][4]
+    float* misc = reinterpret_cast<float*>(smem + kMiscOff);   // scur[4], gate[4]
     const uint16_t* kc = a.k_cur + (size_t)bg * kHeadDim;
     const uint16_t* vc = a.v_cur + (size_t)bg * kHeadDim;
     const float* parts = a.ws + (size_t)bg * n_splits * kPartialFloats;
@@ -504,27 +565,18 @@ int decode_max_splits() { return kMaxSplits; }
 // A fixed 32 MiB array in the library's device image: every GPU that loads
 // the library holds it until the process exits.  Host code must not pass the
 // array's name to a kernel (on the host it is only a stand-in symbol); its
-// device address is looked up once per device with cudaGetSymbolAddress,
-// with that device current, and cached.  All calls on a device share it.
+// device address is looked up with cudaGetSymbolAddress, on every call, in
+// the CUDA context current on the calling thread (so a device reset or a
+// second context on the same device never sees a stale address).  All calls
+// on a device share it.
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticDecodeScratchBytes];
 
 cudaError_t static_decode_scratch(void** ptr) {
-    constexpr int kMaxDevices = 64;
-    static std::mutex mu;
-    static void* addr[kMaxDevices] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        addr[dev] = p;
-    }
-    *ptr = addr[dev];
+    *ptr = p;
     return cudaSuccess;
 }
 

@@ -86,7 +86,7 @@ struct DecodeArgs {
     uint16_t* out;              // [B][G*H][D]
     float* ws;                  // partials [B][G][splits][kPartialFloats]
     int ring_splits, bank_splits;
-    int ring_chunk, bank_chunk; // rows per split (multiples of 4)
+    int ring_chunk, bank_chunk; // rows per split (multiples of 16)
     float qscale;               // softmax_scale * log2(e)
 };
 
@@ -112,7 +112,7 @@ constexpr int kPartialFloats = 4 + 4 + kQPerGroup * kHeadDim;
 
 // Size of the library's own decode scratch (rma_decode_step_noalloc).
 constexpr size_t kStaticDecodeScratchBytes = size_t(32) << 20;
-// Device address of that scratch on the current device (set up on first use per device).
+// Device address of that scratch in the current context (looked up on every call).
 cudaError_t static_decode_scratch(void** ptr);
 
 // Launchers (each returns cudaGetLastError() of its launch).

@@ -143,9 +143,13 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     const uint16_t pair_mask = (uint16_t)(3u << leader);
 
     const int32_t* cnt = S.counters + bg * 4;
-    const int s = max(cnt[0], 0);
-    const int bank_fill = min(max(cnt[1], 0), S.A);
-    const int pend_fill = min(max(cnt[2], 0), S.P);
+    const int c_pos = cnt[0], c_bank = cnt[1], c_pend = cnt[2];
+    if ((c_pos < 0 || c_bank < 0 || c_bank > S.A || c_pend < 0 || c_pend > S.P) && threadIdx.x == 0 && rank == 0 &&
+        blockIdx.x == 0)
+        atomicOr(S.status, (unsigned)RMA_STATUS_BAD_COUNTERS);   // a corrupted state: clamped below
+    const int s = max(c_pos, 0);
+    const int bank_fill = min(max(c_bank, 0), S.A);
+    const int pend_fill = min(max(c_pend, 0), S.P);
     const int fill = min(s, S.R);
 
     // chunks (identical for both CTAs of a pair: tiles 2p and 2p+1 need block chunks 0..p)

@@ -188,9 +188,11 @@ RMA_API int rma_decode_step(rma_state* st, int layer,
  *   Limit: batch * n_groups * (ring_splits + bank_splits) * 4128 bytes must
  *   fit in 32 MiB (batch 512 with the default split shape needs 16.9 MB);
  *   larger calls return RMA_ERR_BUFFER_TOO_SMALL and launch nothing.
- *   The first call on each device looks up the scratch's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   Every call looks up the scratch's device address (cudaGetSymbolAddress)
+ *   in the CUDA context current on the calling thread, so the address is
+ *   never stale after a device reset or in a second context.  The first call
+ *   on a device may load the library's device code there: make that first
+ *   call before any stream capture.
  *   One scratch per GPU is shared by every call on it, and keeps whatever the
  *   last call left: calls that can overlap on the GPU (other streams, other
  *   states) race on it, so the caller must order them.  Nothing in it needs to

@@ -51,6 +51,9 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
             torch.cuda.synchronize()
             err = output_error(to_np(out_na), to_np(out_ws))
             assert err <= TOL, f"call {call} layer {layer}: {err}"
+            # the same kernel, split shape and inputs: the outputs agree bit for bit, so a
+            # partial read from the wrong place or left over from the previous call shows here
+            assert torch.equal(out_na, out_ws), f"call {call} layer {layer}: outputs differ in some bit"
         a, bb = gpu_state_np(st_ws), gpu_state_np(st_na)
         for k in a:
             assert (a[k].tobytes() == bb[k].tobytes()), f"call {call}: state array {k} differs"
