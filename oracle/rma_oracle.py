@@ -307,6 +307,28 @@ def _rank_key(score: float, is_candidate: int, slot: int):
     return (0, -score, is_candidate, slot)
 
 
+def admit_plan(bank_scores, pend_scores, A: int):
+    """The competition of one (sequence, layer, KV group), on scores alone.
+
+    bank_scores: the nb committed anchors' scores (slots 0 .. nb-1); pend_scores:
+    the candidates' (pending slots 0 .. npend-1).  The top min(A, nb + npend)
+    records by the admit order are kept.  Returns (kept count, moves, nan_seen):
+    moves pairs each admitted candidate, in ascending pending slot, with a
+    vacated bank slot (evicted committed slots and empty slots) in ascending
+    order, as (bank slot, pending slot).
+    """
+    nb, npend = len(bank_scores), len(pend_scores)
+    records = ([(float(bank_scores[s]), 0, s) for s in range(nb)] +
+               [(float(pend_scores[t]), 1, t) for t in range(npend)])
+    nan_seen = any(math.isnan(r[0]) for r in records)
+    order = sorted(records, key=lambda r: _rank_key(*r))
+    kept = order[:min(A, len(records))]
+    kept_committed = {slot for (_, kind, slot) in kept if kind == 0}
+    admitted = sorted(slot for (_, kind, slot) in kept if kind == 1)
+    vacated = [s for s in range(nb) if s not in kept_committed] + list(range(nb, A))
+    return len(kept), list(zip(vacated, admitted)), nan_seen
+
+
 def admit(st: State, layer: int, force: bool = False) -> None:
     """Per (sequence, KV group): committed anchors compete with pending candidates.
 
@@ -315,7 +337,7 @@ def admit(st: State, layer: int, force: bool = False) -> None:
     Retained anchors stay in their slots, unchanged ([PRIM] item 3; [CARD]
     "Retained records remain separate and unchanged").  The admitted
     candidates, in ascending pending slot, fill the vacated slots in ascending
-    order.  Afterwards bank_fill = number kept and pend_fill = 0.
+    order (``admit_plan``).  Afterwards bank_fill = number kept and pend_fill = 0.
     """
     cfg = st.cfg
     A, P = cfg.bank_slots, cfg.pend_slots
@@ -325,20 +347,14 @@ def admit(st: State, layer: int, force: bool = False) -> None:
             npend = int(st.pend_fill[layer, b, g])
             if not (npend == P or (force and npend > 0)):
                 continue
-            records = ([(float(st.bank_score[layer, b, g, s]), 0, s) for s in range(nb)] +
-                       [(float(st.pend_score[layer, b, g, t]), 1, t) for t in range(npend)])
-            if any(math.isnan(r[0]) for r in records):
+            kept, moves, nan_seen = admit_plan(st.bank_score[layer, b, g, :nb], st.pend_score[layer, b, g, :npend], A)
+            if nan_seen:
                 st.status |= STATUS_NAN_SCORE
-            order = sorted(records, key=lambda r: _rank_key(*r))
-            kept = order[:min(A, len(records))]
-            kept_committed = {slot for (_, kind, slot) in kept if kind == 0}
-            admitted = sorted(slot for (_, kind, slot) in kept if kind == 1)
-            vacated = [s for s in range(nb) if s not in kept_committed] + list(range(nb, A))
-            for dst, src in zip(vacated, admitted):
+            for dst, src in moves:
                 st.bank_k[layer, b, g, dst] = st.pend_k[layer, b, g, src]
                 st.bank_v[layer, b, g, dst] = st.pend_v[layer, b, g, src]
                 st.bank_score[layer, b, g, dst] = st.pend_score[layer, b, g, src]
-            st.bank_fill[layer, b, g] = len(kept)
+            st.bank_fill[layer, b, g] = kept
             st.pend_fill[layer, b, g] = 0
 
 
