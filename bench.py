@@ -98,18 +98,23 @@ class FillTracker:
     with the method's counter rules: the step reads min(pos, R) ring rows and bank_fill bank rows
     of every group (1 KiB each, K and V), then pos += 1, pend_fill += 1, and a group whose
     pending buffer fills is admitted (bank_fill = min(A, bank_fill + P), pend_fill = 0).
-    Fixed bytes per sequence: q 8,192 + out 8,192 + current K/V 4,096 + ring write 4,096."""
+    Fixed bytes per sequence: q 8,192 + out 8,192 + current K/V 4,096 + ring write 4,096.
+    FP8 storage (fp8=True): a K+V row pair is 2 x 256 code bytes + 2 exponent bytes = 514 bytes,
+    and the ring write stores 4 groups x 514 bytes."""
 
     FIXED = 8192 + 8192 + 4096 + 4096
+    FIXED_FP8 = 8192 + 8192 + 4096 + 4 * 514
 
-    def __init__(self, counters, R: int = 1023, A: int = 1024, P: int = 256):
+    def __init__(self, counters, R: int = 1023, A: int = 1024, P: int = 256, fp8: bool = False):
         c = counters.astype("int64")
         self.pos, self.bank, self.pend = c[..., 0].copy(), c[..., 1].copy(), c[..., 2].copy()
         self.R, self.A, self.P = R, A, P
+        self.row_pair = 514 if fp8 else 1024
+        self.fixed = self.FIXED_FP8 if fp8 else self.FIXED
 
     def launch_bytes(self, layer: int) -> int:
         rows = self.pos[layer].clip(max=self.R) + self.bank[layer]
-        return int(rows.sum() * 1024 + self.pos.shape[1] * self.FIXED)
+        return int(rows.sum() * self.row_pair + self.pos.shape[1] * self.fixed)
 
     def advance(self, layer: int) -> None:
         self.pos[layer] += 1
@@ -196,7 +201,9 @@ class ClockSampler:
 # workload set-up (device side)
 # ---------------------------------------------------------------------------
 
-def make_decode_workload(rma, torch, si, B: int, L: int, kind: str, seed: int, device):
+def make_decode_workload(rma, torch, si, B: int, L: int, kind: str, seed: int, device, fp8: bool = False):
+    """The decode workload's state (BF16; with fp8, the library's quantisation of it into an FP8
+    state, the BF16 one then freed), gate parameters and a pool of 16 step inputs."""
     cfg = rma.Config(batch=B, n_layers=L)
     st = rma.State(cfg, device=device)
     g = torch.Generator(device=device)
@@ -216,6 +223,14 @@ def make_decode_workload(rma, torch, si, B: int, L: int, kind: str, seed: int, d
     cnt[..., 1] = torch.from_numpy(c["bank_fill"])
     cnt[..., 2] = torch.from_numpy(c["pend_fill"])
     st.counters.copy_(cnt)
+    if fp8:
+        cfg8 = rma.Config(batch=B, n_layers=L, kv_format=rma.KV_FP8_E4M3)
+        st8 = rma.State(cfg8, device=device)
+        rma.state_quantize(st8, st)
+        torch.cuda.synchronize(device)
+        del st
+        torch.cuda.empty_cache()
+        cfg, st = cfg8, st8
     w, b = si.gate_params(L, cfg.n_q_heads, cfg.head_dim, seed, device=device)
     pool = [[si.decode_inputs(B, cfg.n_groups, cfg.q_per_group, cfg.head_dim, seed=1000 * s + l, device=device,
                               quantized_scores=(kind == "ragged"))
@@ -370,6 +385,21 @@ def cpu_oracle_prefill_allcores(n_blocks: int = 2) -> dict:
     return {"value": flops / dt / 1e9, "unit": "GFLOP/s", "cores": n, "kind": "oracle",
             "sample": f"{n} sequences (one process per core) x {n_blocks} blocks of 256 tokens at one layer (ring and "
                       f"bank full, forced admits), FP64 numpy oracle; {dt:.1f} s", "cpu": host_cpu()}
+
+
+def all_and_one_core(all_cores, one_core, unit: str) -> dict:
+    """The cpu_baseline object: the oracle on every usable host core (its value and core count),
+    with the one-thread figure beside it.  A failure is reported, never a reason to lose the line."""
+    out = {"value": None, "unit": unit, "cores": _usable_cores(), "kind": "oracle", "sample": "", "cpu": host_cpu()}
+    try:
+        out.update(all_cores())
+    except Exception as ex:
+        out["sample"] = f"all-core run failed: {ex}"
+    try:
+        out["one_core"] = one_core()
+    except Exception as ex:
+        out["one_core"] = {"value": None, "unit": unit, "cores": 1, "sample": f"failed: {ex}"}
+    return out
 
 
 def host_cpu() -> str:
@@ -561,11 +591,8 @@ def run_prefill(args) -> None:
         "gpu_launches": blocks * L,
     }
     if not args.no_cpu_baseline:
-        try:
-            line["cpu_baseline"] = cpu_oracle_prefill()
-        except Exception as ex:   # a report, never a reason to lose the bench line
-            line["cpu_baseline"] = {"value": None, "unit": "GFLOP/s", "cores": 1, "kind": "oracle",
-                                    "sample": f"failed: {ex}"}
+        line["cpu_baseline"] = all_and_one_core(lambda: cpu_oracle_prefill_allcores(n_blocks=16),
+                                                cpu_oracle_prefill, "GFLOP/s")
     print(json.dumps(line), flush=True)
 
 
@@ -716,6 +743,12 @@ def main():
     ap.add_argument("--blocks", type=int, default=128, help="prefill workload: blocks of 256 tokens")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--splits", default=None,
+                    help="decode workloads: ring,bank split counts (rma_set_decode_splits); default: the library's")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="decode workloads: leave rma_set_decode_overlap off (the library default)")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="decode workloads: K/V storage (fp8: E4M3 codes with a per-row scale)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -751,10 +784,17 @@ def main():
     B = args.batch or {"batch": 512, "long": 1, "ragged": 512}[args.workload]
     L = 8
     kind = args.workload
-    cfg, st, w, b, pool = make_decode_workload(rma, torch, si, B, L, kind, seed=rank, device=device)
+    fp8 = args.kv == "fp8"
+    cfg, st, w, b, pool = make_decode_workload(rma, torch, si, B, L, kind, seed=rank, device=device, fp8=fp8)
+    if args.splits:   # before the workspace: its size follows the split shape
+        rs, bs = (int(v) for v in args.splits.split(","))
+        rma.set_decode_splits(st, rs, bs)
     ws = st.workspace(1)
     out = torch.empty(B, 16, 256, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
+    # each launch of a step is another layer: with overlap on, it requests its first ring and bank
+    # tiles while the previous layer's launch finishes (nothing else writes the state in this loop)
+    rma.set_decode_overlap(st, not args.no_overlap)
 
     def step(i, ev=None, strm=None):
         strm = strm if strm is not None else stream
@@ -769,7 +809,7 @@ def main():
 
     # algorithmic bytes of every launch, from the counters the steps will see
     cnt0 = st.counters.cpu().numpy().astype("int64")
-    fills = FillTracker(cnt0)
+    fills = FillTracker(cnt0, fp8=fp8)
     step_bytes = fills.step_bytes
 
     # the long-context case is launch-latency bound: its 8 launches per step are replayed from
@@ -843,7 +883,7 @@ def main():
         durs = [evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(L)]
         dec_ms = sum(durs) / len(durs)
     alg_bytes = sum(timed_bytes) / (K * L)     # per launch, from the exact per-step fills
-    dec_traffic, dec_traffic_note = (profiled_traffic("rma_decode") if kind == "batch"
+    dec_traffic, dec_traffic_note = (profiled_traffic("rma_decode_fp8" if fp8 else "rma_decode") if kind == "batch"
                                      else (None, "captured on the batch-512 workload only"))
     peak, peak_kind = peaks()
 
@@ -915,17 +955,17 @@ def main():
                        "step overlap the kernels of the next"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and kind == "batch":
-        try:
-            cpu = cpu_oracle_decode(n_seq=8, n_layers=8, n_steps=12)
-        except Exception as ex:   # the baseline is a report, never a reason to lose the bench line
-            cpu = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": f"failed: {ex}"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and kind == "batch" and not fp8:
+        cpu = all_and_one_core(lambda: cpu_oracle_decode_allcores(n_steps=64),
+                               lambda: cpu_oracle_decode(n_seq=8, n_layers=8, n_steps=12), UNIT)
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "metric": METRIC + (", FP8 E4M3 K/V storage" if fp8 else ""), "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+            "dtype": "fp8-e4m3 K/V (per-row power-of-two scale), bf16 Q/out" if fp8 else "bf16",
+            "accumulate": "f32", "data": "synthetic",
             "config": {"workload": {"batch": "batch-512 decode: 512 sequences x 8 RMA layers, 4 KV groups x 4 "
                                              "q-heads, head_dim 256, rings full (1023), banks full (1024), pending "
                                              "staggered 0..255 (2 admits per layer per step)",
@@ -933,7 +973,8 @@ def main():
                                             "and bank, pending 0",
                                     "ragged": f"ragged decode: {B} sequences x 8 layers, ring fill U{{1..1023}}, "
                                               "bank fill U{0..1024}, pending U{0..255}, 16-level scores"}[kind],
-                       "batch": B, "layers": L,
+                       "batch": B, "layers": L, "kv_storage": "fp8_e4m3" if fp8 else "bf16",
+                       "decode_overlap": not args.no_overlap, "splits": args.splits or "library default",
                        "step": "8 x rma_decode_step (the admit runs inside the step that fills a pending buffer)",
                        "l2": "inputs larger than L2: the state is %.1f GB" % (st.buffer.numel() / 1e9),
                        "parallelism": f"replicas x{world} (no data-path collective)"},
@@ -946,9 +987,10 @@ def main():
                          "traffic": dec_traffic, "traffic_note": dec_traffic_note,
                          "kernel": "rma_decode (decode_kernel)", "kernel_ms": dec_ms,
                          "algorithmic_bytes_per_launch": alg_bytes,
-                         "algorithmic_bytes_note": "ring min(pos, 1023) + bank_fill rows x 1 KiB per group, plus "
-                                                   "q, out, current K/V and the ring write, from the exact fills of "
-                                                   "every timed launch",
+                         "algorithmic_bytes_note": ("ring min(pos, 1023) + bank_fill rows x " +
+                                                    ("514 B (K and V codes + 2 exponents)" if fp8 else "1 KiB") +
+                                                    " per group, plus q, out, current K/V and the ring write, from the "
+                                                    "exact fills of every timed launch"),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                          else "fallback 6.65 TB/s"},
             "e2e": e2e,

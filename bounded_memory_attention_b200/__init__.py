@@ -26,6 +26,9 @@ STATUS_PREFILL_PENDING_OVERFLOW = 4
 STATUS_BAD_COUNTERS = 8
 STATUS_TIMEOUT = 16
 
+KV_BF16 = 0
+KV_FP8_E4M3 = 1
+
 ERRORS = {0: "RMA_OK", -1: "RMA_ERR_INVALID_ARG", -2: "RMA_ERR_UNSUPPORTED", -3: "RMA_ERR_BUFFER_TOO_SMALL",
           -4: "RMA_ERR_CUDA", -5: "RMA_ERR_MISALIGNED"}
 
@@ -33,13 +36,15 @@ ERRORS = {0: "RMA_OK", -1: "RMA_ERR_INVALID_ARG", -2: "RMA_ERR_UNSUPPORTED", -3:
 class _Config(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("n_groups", ctypes.c_int32),
                 ("q_per_group", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ring_slots", ctypes.c_int32),
-                ("bank_slots", ctypes.c_int32), ("pend_slots", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+                ("bank_slots", ctypes.c_int32), ("pend_slots", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("kv_format", ctypes.c_int32)]
 
 
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "total_bytes", "ring_k", "ring_v", "bank_k", "bank_v", "bank_score",
-        "pend_k", "pend_v", "pend_score", "counters", "tickets", "status")]
+        "pend_k", "pend_v", "pend_score", "counters", "tickets", "status",
+        "ring_k_exp", "ring_v_exp", "bank_k_exp", "bank_v_exp", "pend_k_exp", "pend_v_exp")]
 
 
 def _load():
@@ -66,12 +71,15 @@ def _load():
     lib.rma_admit.argtypes = [vp, i32, i32, vp]
     lib.rma_prefill_block.argtypes = [vp, i32, i32] + [vp] * 10 + [ctypes.c_size_t, vp]
     lib.rma_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.rma_state_quantize.argtypes = [vp, vp, vp]
+    lib.rma_set_decode_overlap.argtypes = [vp, i32]
     lib.rma_strerror.argtypes = [i32]
     lib.rma_strerror.restype = ctypes.c_char_p
     lib.rma_last_error.argtypes = []
     lib.rma_last_error.restype = ctypes.c_char_p
     for f in ("rma_state_alloc", "rma_state_layout", "rma_workspace_bytes", "rma_set_decode_splits",
-              "rma_decode_step", "rma_decode_step_noalloc", "rma_admit", "rma_prefill_block", "rma_get_status"):
+              "rma_decode_step", "rma_decode_step_noalloc", "rma_admit", "rma_prefill_block", "rma_get_status",
+              "rma_state_quantize", "rma_set_decode_overlap"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -93,7 +101,9 @@ def _check(code: int, where: str) -> None:
 
 @dataclass
 class Config:
-    """RMA state dimensions; defaults are the pages' (4 groups, 1,023 + 1 window, 1,024 anchors, 256 pending)."""
+    """RMA state dimensions; defaults are the pages' (4 groups, 1,023 + 1 window, 1,024 anchors, 256 pending).
+
+    kv_format: KV_BF16 (the pages' storage) or KV_FP8_E4M3 (E4M3 codes with a power-of-two scale per row)."""
     batch: int = 1
     n_layers: int = 1
     n_groups: int = 4
@@ -103,10 +113,11 @@ class Config:
     bank_slots: int = 1024
     pend_slots: int = 256
     softmax_scale: float = 1.0 / 16.0
+    kv_format: int = KV_BF16
 
     def _c(self) -> _Config:
         return _Config(self.batch, self.n_layers, self.n_groups, self.q_per_group, self.head_dim,
-                       self.ring_slots, self.bank_slots, self.pend_slots, self.softmax_scale)
+                       self.ring_slots, self.bank_slots, self.pend_slots, self.softmax_scale, self.kv_format)
 
     @property
     def n_q_heads(self) -> int:
@@ -142,6 +153,10 @@ class State:
     Attributes ring_k, ring_v, bank_k, bank_v, bank_score, pend_k, pend_v,
     pend_score and counters are torch views into the buffer with the shapes
     listed in include/rma.h (counters [L, B, G, 4] = pos, bank_fill, pend_fill, 0).
+    In an FP8 state the six K/V views are uint8 E4M3 codes, and ring_k_exp,
+    ring_v_exp, bank_k_exp, bank_v_exp, pend_k_exp, pend_v_exp are int8 views
+    [L, B, G, slots] of the rows' scale exponents (the padding to 16 slots is
+    left out of the view).
     """
 
     def __init__(self, cfg: Config, device=None, stream=None, buffer: torch.Tensor = None):
@@ -179,15 +194,21 @@ class State:
             o = self.layout[name]
             return self.buffer[o:o + nbytes].view(dtype).view(*shape)
 
-        self.ring_k = view("ring_k", torch.bfloat16, (L, B, G, R, D))
-        self.ring_v = view("ring_v", torch.bfloat16, (L, B, G, R, D))
-        self.bank_k = view("bank_k", torch.bfloat16, (L, B, G, A, D))
-        self.bank_v = view("bank_v", torch.bfloat16, (L, B, G, A, D))
+        kv = torch.uint8 if cfg.kv_format == KV_FP8_E4M3 else torch.bfloat16
+        self.ring_k = view("ring_k", kv, (L, B, G, R, D))
+        self.ring_v = view("ring_v", kv, (L, B, G, R, D))
+        self.bank_k = view("bank_k", kv, (L, B, G, A, D))
+        self.bank_v = view("bank_v", kv, (L, B, G, A, D))
         self.bank_score = view("bank_score", torch.float32, (L, B, G, A))
-        self.pend_k = view("pend_k", torch.bfloat16, (L, B, G, P, D))
-        self.pend_v = view("pend_v", torch.bfloat16, (L, B, G, P, D))
+        self.pend_k = view("pend_k", kv, (L, B, G, P, D))
+        self.pend_v = view("pend_v", kv, (L, B, G, P, D))
         self.pend_score = view("pend_score", torch.float32, (L, B, G, P))
         self.counters = view("counters", torch.int32, (L, B, G, 4))
+        if cfg.kv_format == KV_FP8_E4M3:
+            for name, slots in (("ring_k_exp", R), ("ring_v_exp", R), ("bank_k_exp", A), ("bank_v_exp", A),
+                                ("pend_k_exp", P), ("pend_v_exp", P)):
+                padded = (slots + 15) // 16 * 16
+                setattr(self, name, view(name, torch.int8, (L, B, G, padded))[..., :slots])
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -219,6 +240,12 @@ class State:
 
 def set_decode_splits(state: State, ring_splits: int, bank_splits: int) -> None:
     _check(lib.rma_set_decode_splits(state.handle, int(ring_splits), int(bank_splits)), "rma_set_decode_splits")
+
+
+def set_decode_overlap(state: State, enable: bool) -> None:
+    """rma_set_decode_overlap: decode calls stream their ring and bank while the previous decode
+    call on the stream (another layer) finishes; see include/rma.h for the caller's side."""
+    _check(lib.rma_set_decode_overlap(state.handle, 1 if enable else 0), "rma_set_decode_overlap")
 
 
 def decode_step(state: State, layer: int, q, k_cur, v_cur, cand_k, cand_v, cand_score, w_g, b_g, out, ws,
@@ -280,6 +307,11 @@ def prefill_block(state: State, layer: int, q, k, v, cand_k, cand_v, cand_score,
     _check(lib.rma_prefill_block(state.handle, int(layer), int(n), *args, ctypes.c_void_p(ws.data_ptr()),
                                  ws.numel(), _stream_handle(stream)), "rma_prefill_block")
     return out
+
+
+def state_quantize(dst: State, src: State, stream=None) -> None:
+    """rma_state_quantize: every row of the BF16 state `src` quantised into the FP8 state `dst`."""
+    _check(lib.rma_state_quantize(dst.handle, src.handle, _stream_handle(stream)), "rma_state_quantize")
 
 
 def get_status(state: State, stream=None) -> int:

@@ -98,13 +98,43 @@ __device__ __forceinline__ int admit_block_scan(int v, int* warp_tot, int* total
     return r;
 }
 
-// Admit group bg of layer view s with nb committed records and np candidates
-// (both already validated).  Every thread of the CTA (NT of them) must call it; each
-// thread keeps U 16-byte pieces of the row copies in flight;
-// `scratch` is shared memory of admit_scratch_bytes(A, P) bytes, 16-aligned.
-// Writes the bank rows, scores and the counters bank_fill and pend_fill.
-template <int NT, int U = 8>
-__device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t* scratch) {
+// The K and V rows of the admitted candidates: pending slot src[j] -> bank slot dest[j], for
+// j < n_adm, with rows of kChunks 16-byte pieces (32 for BF16, 16 for FP8 codes).
+template <int NT, int U, int kChunks>
+__device__ __forceinline__ void admit_copy_rows(const LayerView& s, int bg, int n_adm, const int* src,
+                                                const int* dest) {
+    constexpr int kRow = kChunks * 16;
+    const uint8_t* pk = reinterpret_cast<const uint8_t*>(s.pend_k) + (size_t)bg * s.P * kRow;
+    const uint8_t* pv = reinterpret_cast<const uint8_t*>(s.pend_v) + (size_t)bg * s.P * kRow;
+    uint8_t* bk = reinterpret_cast<uint8_t*>(s.bank_k) + (size_t)bg * s.A * kRow;
+    uint8_t* bv = reinterpret_cast<uint8_t*>(s.bank_v) + (size_t)bg * s.A * kRow;
+    copy_pieces<NT, U>(n_adm * 2 * kChunks, [&](int e, const uint4*& from_p, uint4*& to_p) {
+        const int j = e / (2 * kChunks);
+        const int c = e % (2 * kChunks);
+        const int from = src[j], to = dest[j];
+        if (c < kChunks) {
+            from_p = reinterpret_cast<const uint4*>(pk + (size_t)from * kRow) + c;
+            to_p = reinterpret_cast<uint4*>(bk + (size_t)to * kRow) + c;
+        } else {
+            from_p = reinterpret_cast<const uint4*>(pv + (size_t)from * kRow) + (c - kChunks);
+            to_p = reinterpret_cast<uint4*>(bv + (size_t)to * kRow) + (c - kChunks);
+        }
+    });
+}
+
+// Where admit_select leaves its result in the scratch: the admitted candidates' pending slots
+// src[j], ascending, and the bank slots they go to, dest[j], ascending, j < n_adm.
+__device__ __forceinline__ int* admit_src(uint8_t* scratch, int A, int P) {
+    return reinterpret_cast<int*>(scratch + ((size_t)(A + P) * 8 + (A + P) + 15) / 16 * 16);
+}
+__device__ __forceinline__ int* admit_dest(uint8_t* scratch, int A, int P) { return admit_src(scratch, A, P) + P; }
+
+// The competition of group bg (nb committed records, np candidates, both validated): every
+// thread of the CTA (NT of them) calls it.  pscore_of(t) is candidate t's score (t < np).
+// Returns n_adm and leaves the lists in the scratch (admit_src / admit_dest); the kept count is
+// min(A, nb + np).  Reads scores only; writes nothing outside the scratch but the status word.
+template <int NT, class PScore>
+__device__ int admit_select(const LayerView& s, int bg, int nb, int np, uint8_t* scratch, PScore pscore_of) {
     const int A = s.A, P = s.P;
     const int tid = threadIdx.x;
     const int n = nb + np;
@@ -126,13 +156,12 @@ __device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t*
     unsigned long long* s_tau = reinterpret_cast<unsigned long long*>(misc + 38);   // 8-aligned
 
     const float* bscore = s.bank_score + (size_t)bg * A;
-    const float* pscore = s.pend_score + (size_t)bg * P;
     if (tid == 0) *s_nan = 0;
     __syncthreads();
     bool nan_seen = false;
     for (int i = tid; i < n; i += NT) {
         const bool committed = i < nb;
-        const float sc = committed ? bscore[i] : pscore[i - nb];
+        const float sc = committed ? bscore[i] : pscore_of(i - nb);
         nan_seen |= isnan(sc);
         keys[i] = admit_key(sc, committed, committed ? i : i - nb);
     }
@@ -238,24 +267,33 @@ __device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t*
         }
     }
     __syncthreads();
+    return n_adm;
+}
 
-    const uint4* pk = reinterpret_cast<const uint4*>(s.pend_k + (size_t)bg * P * kHeadDim);
-    const uint4* pv = reinterpret_cast<const uint4*>(s.pend_v + (size_t)bg * P * kHeadDim);
-    uint4* bk = reinterpret_cast<uint4*>(s.bank_k + (size_t)bg * A * kHeadDim);
-    uint4* bv = reinterpret_cast<uint4*>(s.bank_v + (size_t)bg * A * kHeadDim);
-    constexpr int kChunks = kRowBytes / 16;   // 32 per row
-    copy_pieces<NT, U>(n_adm * 2 * kChunks, [&](int e, const uint4*& from_p, uint4*& to_p) {
-        const int j = e / (2 * kChunks);
-        const int c = e % (2 * kChunks);
-        const int from = src[j], to = dest[j];
-        if (c < kChunks) {
-            from_p = pk + (size_t)from * kChunks + c;
-            to_p = bk + (size_t)to * kChunks + c;
-        } else {
-            from_p = pv + (size_t)from * kChunks + (c - kChunks);
-            to_p = bv + (size_t)to * kChunks + (c - kChunks);
+// Admit group bg of layer view s with nb committed records and np candidates
+// (both already validated).  Every thread of the CTA (NT of them) must call it; each
+// thread keeps U 16-byte pieces of the row copies in flight;
+// `scratch` is shared memory of admit_scratch_bytes(A, P) bytes, 16-aligned.
+// Writes the bank rows, scores and the counters bank_fill and pend_fill.
+template <int NT, int U = 8>
+__device__ void admit_group(const LayerView& s, int bg, int nb, int np, uint8_t* scratch) {
+    const int A = s.A, P = s.P;
+    const int tid = threadIdx.x;
+    const int k = min(A, nb + np);
+    const float* pscore = s.pend_score + (size_t)bg * P;
+    const int n_adm = admit_select<NT>(s, bg, nb, np, scratch, [&](int t) { return pscore[t]; });
+    const int* src = admit_src(scratch, A, P);
+    const int* dest = admit_dest(scratch, A, P);
+
+    if (s.fp8) {
+        admit_copy_rows<NT, U, kHeadDim / 16>(s, bg, n_adm, src, dest);
+        for (int j = tid; j < n_adm; j += NT) {
+            s.bank_ke[(size_t)bg * s.AE + dest[j]] = s.pend_ke[(size_t)bg * s.PE + src[j]];
+            s.bank_ve[(size_t)bg * s.AE + dest[j]] = s.pend_ve[(size_t)bg * s.PE + src[j]];
         }
-    });
+    } else {
+        admit_copy_rows<NT, U, kRowBytes / 16>(s, bg, n_adm, src, dest);
+    }
     for (int j = tid; j < n_adm; j += NT) s.bank_score[(size_t)bg * A + dest[j]] = pscore[src[j]];
     if (tid == 0) {
         int32_t* cnt = s.counters + bg * 4;

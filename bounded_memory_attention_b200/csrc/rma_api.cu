@@ -2,8 +2,11 @@
 // The C declarations and their documentation are in include/rma.h.
 #include <cmath>
 #include <cstdio>
+#include <map>
+#include <mutex>
 #include <new>
 #include <string>
+#include <utility>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -53,12 +56,19 @@ int check_config(const rma_config* c) {
     if (c->bank_slots + c->pend_slots > 4096) return fail(RMA_ERR_UNSUPPORTED, "bank_slots + pend_slots > 4096");
     if (c->batch > 65535 || c->n_groups > 65535) return fail(RMA_ERR_UNSUPPORTED, "batch or n_groups > 65535");
     if ((int64_t)c->batch * c->n_groups > (1 << 24)) return fail(RMA_ERR_UNSUPPORTED, "batch * n_groups > 2^24");
+    if (c->kv_format != RMA_KV_BF16 && c->kv_format != RMA_KV_FP8_E4M3)
+        return fail(RMA_ERR_INVALID_ARG, "kv_format must be RMA_KV_BF16 or RMA_KV_FP8_E4M3");
     return RMA_OK;
 }
 
+// Slot count rounded up to 16: the stride of an FP8 state's exponent arrays, so that the
+// exponents of 16 consecutive rows start on a 16-byte boundary.
+uint64_t pad16(int n) { return round_up((uint64_t)n, 16); }
+
 void compute_layout(const rma_config& c, rma_layout& L) {
     const uint64_t lbg = (uint64_t)c.n_layers * c.batch * c.n_groups;
-    const uint64_t row = (uint64_t)c.head_dim * 2;
+    const bool fp8 = c.kv_format == RMA_KV_FP8_E4M3;
+    const uint64_t row = (uint64_t)c.head_dim * (fp8 ? 1 : 2);
     uint64_t off = 0;
     auto take = [&](uint64_t bytes) {
         const uint64_t o = off;
@@ -76,6 +86,15 @@ void compute_layout(const rma_config& c, rma_layout& L) {
     L.counters = take(lbg * 16);
     L.tickets = take(lbg * 4);
     L.status = take(4);
+    L.ring_k_exp = L.ring_v_exp = L.bank_k_exp = L.bank_v_exp = L.pend_k_exp = L.pend_v_exp = 0;
+    if (fp8) {
+        L.ring_k_exp = take(lbg * pad16(c.ring_slots));
+        L.ring_v_exp = take(lbg * pad16(c.ring_slots));
+        L.bank_k_exp = take(lbg * pad16(c.bank_slots));
+        L.bank_v_exp = take(lbg * pad16(c.bank_slots));
+        L.pend_k_exp = take(lbg * pad16(c.pend_slots));
+        L.pend_v_exp = take(lbg * pad16(c.pend_slots));
+    }
     L.total_bytes = off;
 }
 
@@ -83,14 +102,19 @@ LayerView layer_view(const State& s, int layer) {
     const rma_config& c = s.cfg;
     const uint64_t bg = (uint64_t)c.batch * c.n_groups;
     const uint64_t l = (uint64_t)layer;
+    const bool fp8 = c.kv_format == RMA_KV_FP8_E4M3;
+    const uint64_t rowb = (uint64_t)c.head_dim * (fp8 ? 1 : 2);
+    auto rows = [&](uint64_t off, int slots) {   // layer `layer` of a K/V array (bytes, as uint16_t*)
+        return reinterpret_cast<uint16_t*>(s.base + off + l * bg * slots * rowb);
+    };
     LayerView v;
-    v.ring_k = reinterpret_cast<uint16_t*>(s.base + s.lay.ring_k) + l * bg * c.ring_slots * c.head_dim;
-    v.ring_v = reinterpret_cast<uint16_t*>(s.base + s.lay.ring_v) + l * bg * c.ring_slots * c.head_dim;
-    v.bank_k = reinterpret_cast<uint16_t*>(s.base + s.lay.bank_k) + l * bg * c.bank_slots * c.head_dim;
-    v.bank_v = reinterpret_cast<uint16_t*>(s.base + s.lay.bank_v) + l * bg * c.bank_slots * c.head_dim;
+    v.ring_k = rows(s.lay.ring_k, c.ring_slots);
+    v.ring_v = rows(s.lay.ring_v, c.ring_slots);
+    v.bank_k = rows(s.lay.bank_k, c.bank_slots);
+    v.bank_v = rows(s.lay.bank_v, c.bank_slots);
     v.bank_score = reinterpret_cast<float*>(s.base + s.lay.bank_score) + l * bg * c.bank_slots;
-    v.pend_k = reinterpret_cast<uint16_t*>(s.base + s.lay.pend_k) + l * bg * c.pend_slots * c.head_dim;
-    v.pend_v = reinterpret_cast<uint16_t*>(s.base + s.lay.pend_v) + l * bg * c.pend_slots * c.head_dim;
+    v.pend_k = rows(s.lay.pend_k, c.pend_slots);
+    v.pend_v = rows(s.lay.pend_v, c.pend_slots);
     v.pend_score = reinterpret_cast<float*>(s.base + s.lay.pend_score) + l * bg * c.pend_slots;
     v.counters = reinterpret_cast<int32_t*>(s.base + s.lay.counters) + l * bg * 4;
     v.tickets = reinterpret_cast<uint32_t*>(s.base + s.lay.tickets) + l * bg;
@@ -100,6 +124,19 @@ LayerView layer_view(const State& s, int layer) {
     v.R = c.ring_slots;
     v.A = c.bank_slots;
     v.P = c.pend_slots;
+    v.fp8 = fp8 ? 1 : 0;
+    v.RE = (int)pad16(c.ring_slots);
+    v.AE = (int)pad16(c.bank_slots);
+    v.PE = (int)pad16(c.pend_slots);
+    auto exps = [&](uint64_t off, int stride) {
+        return fp8 ? reinterpret_cast<int8_t*>(s.base + off) + l * bg * stride : nullptr;
+    };
+    v.ring_ke = exps(s.lay.ring_k_exp, v.RE);
+    v.ring_ve = exps(s.lay.ring_v_exp, v.RE);
+    v.bank_ke = exps(s.lay.bank_k_exp, v.AE);
+    v.bank_ve = exps(s.lay.bank_v_exp, v.AE);
+    v.pend_ke = exps(s.lay.pend_k_exp, v.PE);
+    v.pend_ve = exps(s.lay.pend_v_exp, v.PE);
     return v;
 }
 
@@ -136,6 +173,42 @@ Splits decode_splits(const State& s) {
     cut(c.ring_slots, want_r, sp.ring_splits, sp.ring_chunk);
     cut(c.bank_slots, want_b, sp.bank_splits, sp.bank_chunk);
     return sp;
+}
+
+// The kernel this library launched last on each stream (a stream being captured counts as a
+// separate stream per capture), for the decode overlap rule: a decode launch may request its ring
+// and bank before the previous kernel finishes only when that kernel is a decode of another layer
+// (or another state).
+struct LastLaunch {
+    bool decode = false;
+    const void* state = nullptr;
+    int layer = -1;
+};
+std::mutex g_launch_mu;
+std::map<std::pair<uintptr_t, unsigned long long>, LastLaunch> g_last_launch;
+
+std::pair<uintptr_t, unsigned long long> launch_key(cudaStream_t stream) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    unsigned long long id = 0;
+    if (cudaStreamGetCaptureInfo(stream, &st, &id) != cudaSuccess) {
+        (void)cudaGetLastError();
+        id = ~0ull;
+    } else if (st != cudaStreamCaptureStatusActive) {
+        id = 0;
+    }
+    return {reinterpret_cast<uintptr_t>(stream), id};
+}
+
+// Record a launch of this library on `stream` (call with g_launch_mu held).
+void record_launch(const std::pair<uintptr_t, unsigned long long>& key, const LastLaunch& l) {
+    if (g_last_launch.size() > 4096) g_last_launch.clear();   // captures that ended long ago
+    g_last_launch[key] = l;
+}
+
+// A non-decode launch of this library on `stream`.
+void note_other_launch(cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_launch_mu);
+    record_launch(launch_key(stream), LastLaunch{});
 }
 
 State* as_state(rma_state* p) { return reinterpret_cast<State*>(p); }
@@ -182,6 +255,7 @@ int rma_state_alloc(const rma_config* cfg, void* dev_buf, size_t dev_bytes, void
     s->ring_splits_override = 0;
     s->bank_splits_override = 0;
     s->sm_count = sms;
+    s->decode_overlap = 0;
     e = cudaMemsetAsync(s->base + L.counters, 0, L.total_bytes - L.counters, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         delete s;
@@ -262,8 +336,36 @@ int rma_decode_step(rma_state* st, int layer, const uint16_t* q, const uint16_t*
     a.ring_chunk = sp.ring_chunk;
     a.bank_chunk = sp.bank_chunk;
     a.qscale = s->cfg.softmax_scale * 1.4426950408889634f;
-    cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        const auto key = launch_key(cs);
+        a.early = 0;
+        if (s->decode_overlap) {
+            const auto it = g_last_launch.find(key);
+            // the ring and bank of this layer may be read early when the previous kernel on the
+            // stream is a decode of another layer (or another state): it writes nothing of them
+            a.early = (it != g_last_launch.end() && it->second.decode &&
+                       !(it->second.state == s->base && it->second.layer == layer)) ? 1 : 0;
+        }
+        e = launch_decode(a, cs);
+        if (e == cudaSuccess) {
+            LastLaunch l;
+            l.decode = true;
+            l.state = s->base;
+            l.layer = layer;
+            record_launch(key, l);
+        }
+    }
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_decode");
+    return RMA_OK;
+}
+
+int rma_set_decode_overlap(rma_state* st, int enable) {
+    if (!st) return fail(RMA_ERR_INVALID_ARG, "state is NULL");
+    if (enable != 0 && enable != 1) return fail(RMA_ERR_INVALID_ARG, "enable must be 0 or 1");
+    as_state(st)->decode_overlap = enable;
     return RMA_OK;
 }
 
@@ -299,6 +401,7 @@ int rma_admit(rma_state* st, int layer, int force, void* stream) {
     if (force != 0 && force != 1) return fail(RMA_ERR_INVALID_ARG, "force must be 0 or 1");
     cudaError_t e = launch_admit(layer_view(*s, layer), force, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_admit");
+    note_other_launch(static_cast<cudaStream_t>(stream));
     return RMA_OK;
 }
 
@@ -316,6 +419,8 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
         if (!aligned(p, 16)) return fail(RMA_ERR_MISALIGNED, "q, k, v, cand_k, cand_v, w_g, out, ws need 16-byte alignment");
     if (!aligned(cand_score, 4) || !aligned(b_g, 4)) return fail(RMA_ERR_MISALIGNED, "cand_score and b_g need 4-byte alignment");
     if (n_tok < 1) return fail(RMA_ERR_INVALID_ARG, "n_tok must be >= 1");
+    if (s->cfg.kv_format != RMA_KV_BF16)
+        return fail(RMA_ERR_UNSUPPORTED, "rma_prefill_block takes BF16 states (prefill in BF16, then rma_state_quantize)");
     if (n_tok > kMaxPrefillTokens || n_tok > s->cfg.ring_slots)
         return fail(RMA_ERR_UNSUPPORTED, "rma_prefill_block takes n_tok <= 256 and n_tok <= ring_slots");
     if (ws_bytes < prefill_workspace_bytes(s->cfg, n_tok))
@@ -338,6 +443,30 @@ int rma_prefill_block(rma_state* st, int layer, int n_tok, const uint16_t* q, co
     cudaError_t e = launch_prefill(a, cs);
     if (e == cudaErrorNotSupported) return fail(RMA_ERR_UNSUPPORTED, "this prefill block shape is not implemented");
     if (e != cudaSuccess) return cuda_fail(e, "launching rma_prefill_block");
+    note_other_launch(cs);
+    return RMA_OK;
+}
+
+int rma_state_quantize(rma_state* dst, const rma_state* src, void* stream) {
+    NvtxRange range("rma_state_quantize");
+    if (!dst || !src) return fail(RMA_ERR_INVALID_ARG, "dst and src must be non-NULL");
+    State* d = as_state(dst);
+    const State* s = as_state(src);
+    if (d->cfg.kv_format != RMA_KV_FP8_E4M3 || s->cfg.kv_format != RMA_KV_BF16)
+        return fail(RMA_ERR_INVALID_ARG, "rma_state_quantize takes an FP8 destination and a BF16 source");
+    rma_config a = d->cfg, b = s->cfg;
+    a.kv_format = b.kv_format = 0;
+    if (a.batch != b.batch || a.n_layers != b.n_layers || a.n_groups != b.n_groups || a.ring_slots != b.ring_slots ||
+        a.bank_slots != b.bank_slots || a.pend_slots != b.pend_slots)
+        return fail(RMA_ERR_INVALID_ARG, "rma_state_quantize: the two states' dimensions differ");
+    const uint8_t *d0 = d->base, *d1 = d->base + d->lay.total_bytes, *s0 = s->base, *s1 = s->base + s->lay.total_bytes;
+    if (d0 < s1 && s0 < d1) return fail(RMA_ERR_INVALID_ARG, "rma_state_quantize: the two state buffers overlap");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    for (int l = 0; l < d->cfg.n_layers; ++l) {
+        const cudaError_t e = launch_quantize_layer(layer_view(*d, l), layer_view(*s, l), cs);
+        if (e != cudaSuccess) return cuda_fail(e, "launching rma_state_quantize");
+    }
+    note_other_launch(cs);
     return RMA_OK;
 }
 

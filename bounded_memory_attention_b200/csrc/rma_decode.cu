@@ -31,7 +31,22 @@
 //   waiting) merges all partials, adds the current token and the gate, writes
 //   the output and performs the state writes after every read of the step;
 //   when the step fills the pending buffer it also runs the admit for (b, g).
+//
+// FP8 storage (a state with kv_format RMA_KV_FP8_E4M3): the same structure on
+// E4M3 codes and per-row power-of-two scale exponents.  A tile's 16 K rows
+// and 16 V rows (256 bytes each, contiguous in the state) arrive with one bulk
+// copy each, plus one for each set of 16 exponent bytes, two tiles in flight
+// per warp.  The K
+// codes become the FP16 A operand in registers (cvt e4m3x2 -> f16x2, exact);
+// Q is scaled per head by a power of two into FP16 range (exact for every
+// value the FP32 products can resolve); the K exponents scale S per key.  The
+// V codes are converted into an FP16 tile for ldmatrix.trans, and the V
+// exponents fold into P: O is accumulated against its own running maximum of
+// (logit + V exponent), so P V stays in [0, 1] x code range, and is brought
+// back to the softmax's reference at the end.  The ring write and candidate
+// append quantise the rows (one warp per row: amax, exponent, cvt to E4M3).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "rma_admit_impl.cuh"
@@ -47,17 +62,35 @@ constexpr int kTile = 16;                                        // keys per ten
 constexpr int kRowStride = kRowBytes + 16;                       // 528: padded shared-memory row
 constexpr int kSlotBytes = kTile * kRowStride;                   // 8,448: one K or V tile
 constexpr int kWarpRegion = 2 * kSlotBytes;                      // this warp's K slot + V slot
-constexpr int kPipeBytes = kWarps * kWarpRegion;                 // 135,168
 constexpr int kMaxSplits = 64;                                   // ring_splits + bank_splits
-constexpr int kCoefOff = kPipeBytes;                             // [(kMaxSplits + 1)][4] floats
-constexpr int kMiscOff = kCoefOff + (kMaxSplits + 1) * 4 * 4;    // scur[4], gate[4] (+ pad)
-constexpr int kBarOff = kMiscOff + 16 * 4;                       // [kWarps][2] mbarriers
-constexpr int kSmemBytes = kBarOff + kWarps * 2 * 8;
+// FP8 storage, per warp: two stages of (K codes + exponents, V codes + exponents), then the FP16 V tile.
+// A tile's 16 code rows are contiguous in the state, so each slot arrives with one bulk copy for
+// the codes and one for the exponents (four requests per tile, not one per row).
+constexpr int kF8Hdr = 64;                                       // a slot's 16 exponent bytes (+ pad)
+constexpr int kF8Row = kHeadDim;                                 // 256 code bytes per row, unpadded
+constexpr int kF8KSlot = kF8Hdr + kTile * kF8Row;                // 4,160
+constexpr int kF8VSlot = kF8Hdr + kTile * kF8Row;                // 4,160
+constexpr int kF8Stage = kF8KSlot + kF8VSlot;                    // 8,320
+constexpr int kF8Stages = 2;
+constexpr int kF8WarpRegion = kF8Stages * kF8Stage + kSlotBytes; // 25,088
+
+// Shared-memory layout of a storage: the warps' regions, the merge's coefficients and scalars, mbarriers.
+template <bool kFp8>
+struct Smem {
+    static constexpr int kRegion = kFp8 ? kF8WarpRegion : kWarpRegion;
+    static constexpr int kPipe = kWarps * kRegion;
+    static constexpr int kCoef = kPipe;                          // [(kMaxSplits + 1)][4] floats
+    static constexpr int kMisc = kCoef + (kMaxSplits + 1) * 4 * 4;   // scur[4], gate[4] (+ pad)
+    static constexpr int kBars = kMisc + 16 * 4;                 // [kWarps][2 or 4] mbarriers
+    static constexpr int kNumBars = kWarps * (kFp8 ? 4 : 2);
+    static constexpr int kBytes = kBars + kNumBars * 8;
+    static_assert(kRegion >= kPartialFloats * 4, "a warp's region must hold one warp partial");
+    static_assert(kPipe >= (int)admit_scratch_bytes(1, 4095), "the admit reuses the pipeline region (any A + P <= 4096)");
+    static_assert((kBars & 7) == 0, "mbarriers are 8-byte aligned");
+    static_assert(kBytes <= 227 * 1024, "shared memory per CTA");
+};
 
 static_assert(kWarps == 8, "merger assigns 8 dot products to 8 warps");
-static_assert(kSlotBytes >= kPartialFloats * 4, "a warp's K slot must hold one warp partial");
-static_assert(kPipeBytes >= (int)admit_scratch_bytes(1, 4095), "the admit reuses the pipeline region (any A + P <= 4096)");
-static_assert((kBarOff & 7) == 0, "mbarriers are 8-byte aligned");
 
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -78,6 +111,12 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     uint4 r;
     asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];\n"
                  : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];\n" : "=r"(r.x), "=r"(r.y) : "l"(p));
     return r;
 }
 
@@ -114,13 +153,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Transpose an 8x8 matrix of 16-bit values held one row pair per lane in the mma fragment layout.
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-    return y;
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -133,6 +165,81 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// D (16x8 FP32) += A (16x16 FP16, row) . B (16x8 FP16, col)
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (low byte first) -> two FP16 values (low half first); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t r;
+    const unsigned short v = (unsigned short)(two_codes & 0xffffu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(r) : "h"(v));
+    return r;
+}
+
+// Two FP32 values -> two E4M3 codes (lo in the low byte), round to nearest even (|x| <= 448 here).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 2^e as FP32 for e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2i(int e) {
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u >> (-127 - e));
+}
+
+// The scale exponent of an FP8 row: the smallest e in [-127, 127] with amax <= 448 * 2^e (0 for
+// amax == 0).  With amax = 1.M * 2^(E - 127) and 448 = 1.75 * 2^8: e = E - 135, plus one when
+// 1.M > 1.75 (M > 0x600000); amax below the normal range gives -127.
+__device__ __forceinline__ int fp8_row_exponent(float amax) {
+    if (amax == 0.f) return 0;
+    const uint32_t u = __float_as_uint(amax);
+    const int E = (int)(u >> 23);
+    if (E == 0) return -127;
+    return max(-127, min(127, E - 135 + ((u & 0x7FFFFFu) > 0x600000u ? 1 : 0)));
+}
+
+// Quantise one BF16 row of 256 values (a warp: lane L takes values 8 L .. 8 L + 7) into 256
+// E4M3 codes at dst and its scale exponent at *dexp.
+__device__ __forceinline__ void quantize_row_warp(const uint16_t* src, uint8_t* dst, int8_t* dexp, int lane) {
+    const uint4 r = ld_nc_v4(src + lane * 8);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    float f[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        f[2 * k] = __uint_as_float(w[k] << 16);
+        f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+    float am = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) am = fmaxf(am, fabsf(f[k]));
+    am = warp_max(am);
+    const int e = fp8_row_exponent(am);
+    const float sc = pow2i(-e);   // an exact power-of-two scaling
+    const uint32_t lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | (f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16);
+    const uint32_t hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | (f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16);
+    *reinterpret_cast<uint2*>(dst + lane * 8) = make_uint2(lo, hi);
+    if (lane == 0) *dexp = (int8_t)e;
+}
+
+// Transpose an 8x8 matrix of 16-bit values held one row pair per lane in the mma fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ float dot8(const float2 (&q)[4], const uint4& k) {
     float2 d = __fmul2_rn(q[0], bf2_to_f2(k.x));
     d = __ffma2_rn(q[1], bf2_to_f2(k.y), d);
@@ -140,6 +247,11 @@ __device__ __forceinline__ float dot8(const float2 (&q)[4], const uint4& k) {
     d = __ffma2_rn(q[3], bf2_to_f2(k.w), d);
     return d.x + d.y;
 }
+
+// Programmatic dependent launch: wait until the previous kernel in the stream has completed and
+// its writes are visible; let the next kernel's CTAs be scheduled.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 // Bounded wait on an mbarrier phase (about two seconds); on timeout sets RMA_STATUS_TIMEOUT and
 // returns false.
@@ -155,49 +267,13 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint3
     return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = a.s.G;
-    const int bg = b * G + g;
-    const int n_splits = a.ring_splits + a.bank_splits;
-
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
-    if (tid < 2 * kWarps) ptx::mbar_init(&bars[tid], 1);
-    ptx::fence_mbar_init();
-
-    const int32_t* cnt = a.s.counters + bg * 4;
-    int pos = cnt[0], bank_fill = cnt[1], pend_fill = cnt[2];
-    if (pos < 0 || bank_fill < 0 || bank_fill > a.s.A || pend_fill < 0 || pend_fill > a.s.P) {
-        // a corrupted state: never index outside the buffers
-        if (threadIdx.x == 0 && split == 0) atomicOr(a.s.status, (unsigned)RMA_STATUS_BAD_COUNTERS);
-        pos = max(pos, 0);
-        bank_fill = min(max(bank_fill, 0), a.s.A);
-        pend_fill = min(max(pend_fill, 0), a.s.P);
-    }
-
-    // ---- this CTA's row range ----
-    const bool is_bank = split >= a.ring_splits;
-    int nrows;
-    const uint16_t* kbase;
-    const uint16_t* vbase;
-    if (!is_bank) {
-        const int fill = min(pos, a.s.R);
-        const int row0 = split * a.ring_chunk;
-        nrows = max(0, min(a.ring_chunk, fill - row0));
-        const size_t off = ((size_t)bg * a.s.R + row0) * kHeadDim;
-        kbase = a.s.ring_k + off;
-        vbase = a.s.ring_v + off;
-    } else {
-        const int row0 = (split - a.ring_splits) * a.bank_chunk;
-        nrows = max(0, min(a.bank_chunk, bank_fill - row0));
-        const size_t off = ((size_t)bg * a.s.A + row0) * kHeadDim;
-        kbase = a.s.bank_k + off;
-        vbase = a.s.bank_v + off;
-    }
-    __syncthreads();   // the mbarriers are initialised
-
+// BF16 storage: stream this warp's tiles of the CTA's row range and leave the warp's running
+// softmax of heads 2 tq and 2 tq + 1 (lanes with tq >= 2 carry the unused columns) in m0, m1,
+// l0, l1 (row sums already reduced over the fragment's key rows) and acc (O^T fragments).
+__device__ __forceinline__ void stream_bf16(const DecodeArgs& a, uint8_t* smem, uint64_t* bars, int warp, int lane,
+                                            int nrows, const uint16_t* kbase, const uint16_t* vbase,
+                                            const uint16_t* qg, float& m0, float& m1, float& l0, float& l1,
+                                            float (&acc)[16][4]) {
     // ---- this warp's tiles: w, w + 8, ...; K slot and V slot, one mbarrier each ----
     uint8_t* wsm = smem + warp * kWarpRegion;
     const uint32_t kslot = ptx::smem_u32(wsm), vslot = kslot + kSlotBytes;
@@ -221,12 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         issue(0, false);
         issue(0, true);
     }
+    if (a.early) {   // the first tile is requested: now wait for the previous kernel (see decode_kernel)
+        grid_dep_wait();
+        grid_dep_launch();
+    }
 
     // ---- Q^T fragments (the B operand of S^T = K Q^T), loaded while the first tiles are in flight:
     //      lane (gq = lane / 4, tq = lane % 4) holds head gq's dims 16 c + 2 tq (+1) and 16 c + 2 tq + 8 (+9);
     //      heads 4..7 of the 8 columns are zero ----
     const int gq = lane >> 2, tq = lane & 3;
-    const uint16_t* qg = a.q + ((size_t)b * G * kQPerGroup + (size_t)g * kQPerGroup) * kHeadDim;
     uint32_t qf[16][2];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
@@ -241,11 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // V^T (A operand via .trans, rows = dims): matrices (dims +0-7 | +8-15) x (keys 0-7 | 8-15)
     const uint32_t v_addr = vslot + (uint32_t)((lr + 8 * (lm >> 1)) * kRowStride + 16 * (lm & 1));
 
-    // running softmax of heads 2 tq and 2 tq + 1 (lanes with tq >= 2 carry the unused columns)
-    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
-    float acc[16][4];
-#pragma unroll
-    for (int mt = 0; mt < 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     const float qs = a.qscale;
     bool ok = true;
     int k_issued = my_n > 0 ? 1 : 0, v_issued = k_issued;
@@ -338,6 +412,283 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
 
+}
+
+// FP8 storage: the same contract as stream_bf16 on E4M3 codes with per-row scale exponents
+// (kexp / vexp: the exponents of the range's rows, 16-byte aligned).
+__device__ __forceinline__ void stream_fp8(const DecodeArgs& a, uint8_t* smem, uint64_t* bars, int warp, int lane,
+                                           int nrows, const uint8_t* kcodes, const uint8_t* vcodes,
+                                           const int8_t* kexp, const int8_t* vexp, const uint16_t* qg, float& m0,
+                                           float& m1, float& l0, float& l1, float (&acc)[16][4]) {
+    uint8_t* wsm = smem + warp * kF8WarpRegion;
+    uint8_t* vt = wsm + kF8Stages * kF8Stage;      // the FP16 V tile (16 rows x 528 bytes)
+    uint64_t* kb = &bars[4 * warp];                // K of stage 0 / 1
+    uint64_t* vb = &bars[4 * warp + 2];            // V of stage 0 / 1
+    const int n_tiles = (nrows + kTile - 1) / kTile;
+    const int my_n = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
+
+    // tile i of this warp -> stage i & 1: lane 0 copies its K code rows (one contiguous range) and
+    // the 16 K exponents, lane 16 its V code rows and V exponents
+    auto issue = [&](int i) {
+        const int st = i & 1;
+        const int r0 = (warp + i * kWarps) * kTile;
+        const int nv = min(kTile, nrows - r0);
+        uint8_t* ks = wsm + st * kF8Stage;
+        uint8_t* vs = ks + kF8KSlot;
+        if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(&kb[st], (uint32_t)(nv * kF8Row + 16));
+            bulk_g2s(ptx::smem_u32(ks + kF8Hdr), kcodes + (size_t)r0 * kF8Row, (uint32_t)(nv * kF8Row),
+                     ptx::smem_u32(&kb[st]));
+            bulk_g2s(ptx::smem_u32(ks), kexp + r0, 16, ptx::smem_u32(&kb[st]));
+        } else if (lane == 16) {
+            ptx::mbar_arrive_expect_tx(&vb[st], (uint32_t)(nv * kF8Row + 16));
+            bulk_g2s(ptx::smem_u32(vs + kF8Hdr), vcodes + (size_t)r0 * kF8Row, (uint32_t)(nv * kF8Row),
+                     ptx::smem_u32(&vb[st]));
+            bulk_g2s(ptx::smem_u32(vs), vexp + r0, 16, ptx::smem_u32(&vb[st]));
+        }
+        __syncwarp();
+    };
+    if (my_n > 0) issue(0);
+    if (my_n > 1) issue(1);
+    int issued = min(my_n, 2);
+    if (a.early) {   // the first tiles are requested: now wait for the previous kernel (see decode_kernel)
+        grid_dep_wait();
+        grid_dep_launch();
+    }
+
+    // ---- Q^T fragments in FP16.  Chunk c = 4 j + i of the contraction takes, for lane (gq, tq),
+    //      dims 64 j + 16 tq + 4 i + {0, 1} as k = 2 tq, 2 tq + 1 and + {2, 3} as k = 2 tq + 8, 2 tq + 9
+    //      (the K fragments below use the same order), so that each lane reads its K bytes with
+    //      16-byte loads.  Head gq's values are scaled by 2^-eq, eq putting its largest magnitude
+    //      in [2^14, 2^15); the logits take 2^eq back. ----
+    const int gq = lane >> 2, tq = lane & 3;
+    uint2 qraw[16];
+    float am = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        qraw[c] = gq < kQPerGroup ? ld_nc_v2(qg + gq * kHeadDim + 64 * (c >> 2) + 16 * tq + 4 * (c & 3))
+                                  : make_uint2(0u, 0u);
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(__uint_as_float(qraw[c].x << 16)), fabsf(__uint_as_float(qraw[c].x & 0xffff0000u))),
+                             fmaxf(fabsf(__uint_as_float(qraw[c].y << 16)), fabsf(__uint_as_float(qraw[c].y & 0xffff0000u)))));
+    }
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    const int eq = am == 0.f ? 0 : max(-126, min(126, (int)(__float_as_uint(am) >> 23) - 141));
+    const float qsc = pow2i(-eq);
+    uint32_t qf[16][2];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        qf[c][0] = pack_f16(__uint_as_float(qraw[c].x << 16) * qsc, __uint_as_float(qraw[c].x & 0xffff0000u) * qsc);
+        qf[c][1] = pack_f16(__uint_as_float(qraw[c].y << 16) * qsc, __uint_as_float(qraw[c].y & 0xffff0000u) * qsc);
+    }
+    // logit scale of this lane's S^T columns (heads 2 tq, 2 tq + 1; their Q lives in lanes 8 tq, 8 tq + 4)
+    const float qs0 = a.qscale * pow2i(__shfl_sync(0xffffffffu, eq, (8 * tq) & 31));
+    const float qs1 = a.qscale * pow2i(__shfl_sync(0xffffffffu, eq, (8 * tq + 4) & 31));
+
+    const int lr = lane & 7, lm = lane >> 3;
+    const uint32_t v_addr = ptx::smem_u32(vt) + (uint32_t)((lr + 8 * (lm >> 1)) * kRowStride + 16 * (lm & 1));
+    // O is accumulated against its own reference n (running max of logit + V exponent)
+    float n0 = -CUDART_INF_F, n1 = -CUDART_INF_F;
+    bool ok = true;
+    int i = 0;
+    for (; i < my_n; ++i) {
+        const int st = i & 1;
+        const uint32_t par = (i >> 1) & 1;
+        const int r0 = (warp + i * kWarps) * kTile;
+        const int nv = min(kTile, nrows - r0);
+        uint8_t* ks = wsm + st * kF8Stage;
+        uint8_t* vs = ks + kF8KSlot;
+        // ---- S^T = K Q^T on the codes: 16 FP16 MMAs in four chains ----
+        if (!wait_phase(&kb[st], par, a.s.status)) { ok = false; break; }
+        float s[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) s[c][0] = s[c][1] = s[c][2] = s[c][3] = 0.f;
+        const uint8_t* klo = ks + kF8Hdr + gq * kF8Row + 16 * tq;
+        const uint8_t* khi = klo + 8 * kF8Row;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 ra = *reinterpret_cast<const uint4*>(klo + 64 * j);
+            const uint4 rb = *reinterpret_cast<const uint4*>(khi + 64 * j);
+            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+                uint32_t af[4];
+                af[0] = e4m3x2_to_f16x2(wa[i4]);
+                af[1] = e4m3x2_to_f16x2(wb[i4]);
+                af[2] = e4m3x2_to_f16x2(wa[i4] >> 16);
+                af[3] = e4m3x2_to_f16x2(wb[i4] >> 16);
+                mma_16816_f16(s[i4], af, qf[4 * j + i4][0], qf[4 * j + i4][1]);
+            }
+        }
+        const float ks_lo = pow2i((int)(int8_t)ks[gq]), ks_hi = pow2i((int)(int8_t)ks[gq + 8]);
+        // ---- logits x (log2 domain): (key gq | gq + 8) x (head 2 tq | 2 tq + 1); the softmax sums l ----
+        const bool va = gq < nv, vb2 = gq + 8 < nv;
+        const float x0 = va ? (((s[0][0] + s[1][0]) + (s[2][0] + s[3][0])) * qs0) * ks_lo : -CUDART_INF_F;
+        const float x1 = va ? (((s[0][1] + s[1][1]) + (s[2][1] + s[3][1])) * qs1) * ks_lo : -CUDART_INF_F;
+        const float x2 = vb2 ? (((s[0][2] + s[1][2]) + (s[2][2] + s[3][2])) * qs0) * ks_hi : -CUDART_INF_F;
+        const float x3 = vb2 ? (((s[0][3] + s[1][3]) + (s[2][3] + s[3][3])) * qs1) * ks_hi : -CUDART_INF_F;
+        float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, o));
+            t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, o));
+        }
+        if (t0 > m0) {
+            l0 *= (m0 == -CUDART_INF_F) ? 0.f : fast_ex2(m0 - t0);
+            m0 = t0;
+        }
+        if (t1 > m1) {
+            l1 *= (m1 == -CUDART_INF_F) ? 0.f : fast_ex2(m1 - t1);
+            m1 = t1;
+        }
+        l0 += fast_ex2(x0 - m0) + fast_ex2(x2 - m0);
+        l1 += fast_ex2(x1 - m1) + fast_ex2(x3 - m1);
+        // ---- V codes -> the FP16 tile (rows past the range become zero); the stage is then free ----
+        if (!wait_phase(&vb[st], par, a.s.status)) { ok = false; break; }
+        const float ev_lo = (float)(int8_t)vs[gq], ev_hi = (float)(int8_t)vs[gq + 8];
+        {
+            // pass k: the warp reads 512 contiguous code bytes (rows 2k and 2k + 1), lane L the 16
+            // codes at columns 16 (L % 16) of row 2k + L / 16
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int vr = 2 * k + (lane >> 4), col = 16 * (lane & 15);
+                const uint4 u = vr < nv ? *reinterpret_cast<const uint4*>(vs + kF8Hdr + vr * kF8Row + col)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                uint8_t* dst = vt + vr * kRowStride + 2 * col;
+                *reinterpret_cast<uint4*>(dst) = make_uint4(e4m3x2_to_f16x2(u.x), e4m3x2_to_f16x2(u.x >> 16),
+                                                            e4m3x2_to_f16x2(u.y), e4m3x2_to_f16x2(u.y >> 16));
+                *reinterpret_cast<uint4*>(dst + 16) = make_uint4(e4m3x2_to_f16x2(u.z), e4m3x2_to_f16x2(u.z >> 16),
+                                                                 e4m3x2_to_f16x2(u.w), e4m3x2_to_f16x2(u.w >> 16));
+            }
+        }
+        __syncwarp();
+        if (i + 2 < my_n) {   // both slots of this stage have been read: request tile i + 2
+            issue(i + 2);
+            ++issued;
+        }
+        // ---- P' = 2^(x + V exponent - n), O^T += V^T P'^T on the codes ----
+        const float y0 = x0 + ev_lo, y1 = x1 + ev_lo, y2 = x2 + ev_hi, y3 = x3 + ev_hi;
+        float u0 = fmaxf(y0, y2), u1 = fmaxf(y1, y3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            u0 = fmaxf(u0, __shfl_xor_sync(0xffffffffu, u0, o));
+            u1 = fmaxf(u1, __shfl_xor_sync(0xffffffffu, u1, o));
+        }
+        const bool up0 = u0 > n0, up1 = u1 > n1;
+        if (__any_sync(0xffffffffu, up0 || up1)) {
+            const float f0 = up0 ? (n0 == -CUDART_INF_F ? 0.f : fast_ex2(n0 - u0)) : 1.f;
+            const float f1 = up1 ? (n1 == -CUDART_INF_F ? 0.f : fast_ex2(n1 - u1)) : 1.f;
+            n0 = up0 ? u0 : n0;
+            n1 = up1 ? u1 : n1;
+#pragma unroll
+            for (int mt = 0; mt < 16; ++mt) {
+                acc[mt][0] *= f0;
+                acc[mt][1] *= f1;
+                acc[mt][2] *= f0;
+                acc[mt][3] *= f1;
+            }
+        }
+        const uint32_t pb0 = movmatrix_trans(pack_f16(fast_ex2(y0 - n0), fast_ex2(y1 - n1)));
+        const uint32_t pb1 = movmatrix_trans(pack_f16(fast_ex2(y2 - n0), fast_ex2(y3 - n1)));
+#pragma unroll
+        for (int mt = 0; mt < 16; ++mt) {
+            uint32_t af[4];
+            ldsm_x4_trans(v_addr + 32 * mt, af);
+            mma_16816_f16(acc[mt], af, pb0, pb1);
+        }
+        __syncwarp();   // the FP16 tile has been read before the next tile's conversion
+    }
+    if (!ok) {
+        // a wait ran out: let every copy this warp requested land before its slots are reused
+        for (int t = i; t < issued; ++t) {
+            wait_phase(&kb[t & 1], (t >> 1) & 1, a.s.status);
+            wait_phase(&vb[t & 1], (t >> 1) & 1, a.s.status);
+        }
+    }
+    // O back to the softmax's reference: acc = O * 2^(n - m)
+    const float f0 = (m0 == -CUDART_INF_F) ? 0.f : fast_ex2(n0 - m0);
+    const float f1 = (m1 == -CUDART_INF_F) ? 0.f : fast_ex2(n1 - m1);
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+        acc[mt][0] *= f0;
+        acc[mt][1] *= f1;
+        acc[mt][2] *= f0;
+        acc[mt][3] *= f1;
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+    using L = Smem<kFp8>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = a.s.G;
+    const int bg = b * G + g;
+    const int n_splits = a.ring_splits + a.bank_splits;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    if (tid < L::kNumBars) ptx::mbar_init(&bars[tid], 1);
+    ptx::fence_mbar_init();
+
+    // The launch may begin before the previous kernel in the stream has finished.  By default
+    // nothing in global memory is touched before that kernel has completed.  With `early` (the host
+    // found that kernel to be a decode of this library on another layer or another state) the
+    // counters are read and the first ring / bank tiles requested first, and the wait comes before
+    // anything else is read or written (the inputs come after it, whoever produced them).  Either
+    // way this launch lets its own dependents start only after its wait, so a launch never overlaps
+    // more than the one before it.
+    if (!a.early) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
+
+    const int32_t* cnt = a.s.counters + bg * 4;
+    int pos = cnt[0], bank_fill = cnt[1], pend_fill = cnt[2];
+    if (pos < 0 || bank_fill < 0 || bank_fill > a.s.A || pend_fill < 0 || pend_fill > a.s.P) {
+        // a corrupted state: never index outside the buffers
+        if (threadIdx.x == 0 && split == 0) atomicOr(a.s.status, (unsigned)RMA_STATUS_BAD_COUNTERS);
+        pos = max(pos, 0);
+        bank_fill = min(max(bank_fill, 0), a.s.A);
+        pend_fill = min(max(pend_fill, 0), a.s.P);
+    }
+
+    // ---- this CTA's row range: rows [row0, row0 + nrows) of the ring or the bank ----
+    const bool is_bank = split >= a.ring_splits;
+    int nrows, row0;
+    if (!is_bank) {
+        row0 = split * a.ring_chunk;
+        nrows = max(0, min(a.ring_chunk, min(pos, a.s.R) - row0));
+    } else {
+        row0 = (split - a.ring_splits) * a.bank_chunk;
+        nrows = max(0, min(a.bank_chunk, bank_fill - row0));
+    }
+    const size_t row_index = (size_t)bg * (is_bank ? a.s.A : a.s.R) + row0;
+    __syncthreads();   // the mbarriers are initialised
+
+    const uint16_t* qg = a.q + ((size_t)b * G * kQPerGroup + (size_t)g * kQPerGroup) * kHeadDim;
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    float acc[16][4];
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    if constexpr (kFp8) {
+        const uint8_t* kc8 = reinterpret_cast<const uint8_t*>(is_bank ? a.s.bank_k : a.s.ring_k) + row_index * kHeadDim;
+        const uint8_t* vc8 = reinterpret_cast<const uint8_t*>(is_bank ? a.s.bank_v : a.s.ring_v) + row_index * kHeadDim;
+        const size_t erow = (size_t)bg * (is_bank ? a.s.AE : a.s.RE) + row0;
+        stream_fp8(a, smem, bars, warp, lane, nrows, kc8, vc8, (is_bank ? a.s.bank_ke : a.s.ring_ke) + erow,
+                   (is_bank ? a.s.bank_ve : a.s.ring_ve) + erow, qg, m0, m1, l0, l1, acc);
+    } else {
+        stream_bf16(a, smem, bars, warp, lane, nrows, (is_bank ? a.s.bank_k : a.s.ring_k) + row_index * kHeadDim,
+                    (is_bank ? a.s.bank_v : a.s.ring_v) + row_index * kHeadDim, qg, m0, m1, l0, l1, acc);
+    }
+    const int gq = lane >> 2, tq = lane & 3;
+    uint8_t* wsm = smem + warp * L::kRegion;
+
     // ---- this warp's partial (m, l, acc) into its K slot: lanes with tq < 2 hold heads 0..3 ----
     __syncwarp();
     float* wpart = reinterpret_cast<float*>(wsm);
@@ -367,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         float M = -CUDART_INF_F;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            mw[w] = reinterpret_cast<const float*>(smem + w * kWarpRegion)[h];
+            mw[w] = reinterpret_cast<const float*>(smem + w * L::kRegion)[h];
             M = fmaxf(M, mw[w]);
         }
         const float Mu = (M == -CUDART_INF_F) ? 0.f : M;
@@ -375,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         float L = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float* wp = reinterpret_cast<const float*>(smem + w * kWarpRegion);
+            const float* wp = reinterpret_cast<const float*>(smem + w * L::kRegion);
             const float c = fast_ex2(mw[w] - Mu);
             L += c * wp[4 + h];
             const float4 v = *reinterpret_cast<const float4*>(wp + 8 + h * kHeadDim + d);
@@ -400,8 +751,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     __threadfence();
 
     // ---- last CTA of (b, g): merge every split, add the current token, gate, write ----
-    float* coef = reinterpret_cast<float*>(smem + kCoefOff);   // [(n_splits+1)][4]
-    float* misc = reinterpret_cast<float*>(smem + kMiscOff);   // scur[4], gate[4]
+    float* coef = reinterpret_cast<float*>(smem + L::kCoef);   // [(n_splits+1)][4]
+    float* misc = reinterpret_cast<float*>(smem + L::kMisc);   // scur[4], gate[4]
     const uint16_t* kc = a.k_cur + (size_t)bg * kHeadDim;
     const uint16_t* vc = a.v_cur + (size_t)bg * kHeadDim;
     const float* parts = a.ws + (size_t)bg * n_splits * kPartialFloats;
@@ -515,21 +866,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // ---- state writes: every split of (b, g) has finished reading ----
     const int slot = pos % a.s.R;
     const bool room = pend_fill < a.s.P;
-    if (tid < 32) {
-        reinterpret_cast<uint4*>(a.s.ring_k + ((size_t)bg * a.s.R + slot) * kHeadDim)[lane] =
-            ld_nc_v4(kc + lane * 8);
-    } else if (tid < 64) {
-        reinterpret_cast<uint4*>(a.s.ring_v + ((size_t)bg * a.s.R + slot) * kHeadDim)[lane] =
-            ld_nc_v4(vc + lane * 8);
-    } else if (tid < 96) {
-        if (room)
-            reinterpret_cast<uint4*>(a.s.pend_k + ((size_t)bg * a.s.P + pend_fill) * kHeadDim)[lane] =
-                ld_nc_v4(a.cand_k + (size_t)bg * kHeadDim + lane * 8);
-    } else if (tid < 128) {
-        if (room)
-            reinterpret_cast<uint4*>(a.s.pend_v + ((size_t)bg * a.s.P + pend_fill) * kHeadDim)[lane] =
-                ld_nc_v4(a.cand_v + (size_t)bg * kHeadDim + lane * 8);
-    } else if (tid == 128) {
+    if constexpr (kFp8) {
+        // one warp per row: quantise into codes and a scale exponent
+        uint8_t* rk = reinterpret_cast<uint8_t*>(a.s.ring_k) + ((size_t)bg * a.s.R + slot) * kHeadDim;
+        uint8_t* rv = reinterpret_cast<uint8_t*>(a.s.ring_v) + ((size_t)bg * a.s.R + slot) * kHeadDim;
+        uint8_t* pk = reinterpret_cast<uint8_t*>(a.s.pend_k) + ((size_t)bg * a.s.P + pend_fill) * kHeadDim;
+        uint8_t* pv = reinterpret_cast<uint8_t*>(a.s.pend_v) + ((size_t)bg * a.s.P + pend_fill) * kHeadDim;
+        if (warp == 0) {
+            quantize_row_warp(kc, rk, a.s.ring_ke + (size_t)bg * a.s.RE + slot, lane);
+        } else if (warp == 1) {
+            quantize_row_warp(vc, rv, a.s.ring_ve + (size_t)bg * a.s.RE + slot, lane);
+        } else if (warp == 2) {
+            if (room) quantize_row_warp(a.cand_k + (size_t)bg * kHeadDim, pk, a.s.pend_ke + (size_t)bg * a.s.PE + pend_fill, lane);
+        } else if (warp == 3) {
+            if (room) quantize_row_warp(a.cand_v + (size_t)bg * kHeadDim, pv, a.s.pend_ve + (size_t)bg * a.s.PE + pend_fill, lane);
+        }
+    } else {
+        if (tid < 32) {
+            reinterpret_cast<uint4*>(a.s.ring_k + ((size_t)bg * a.s.R + slot) * kHeadDim)[lane] =
+                ld_nc_v4(kc + lane * 8);
+        } else if (tid < 64) {
+            reinterpret_cast<uint4*>(a.s.ring_v + ((size_t)bg * a.s.R + slot) * kHeadDim)[lane] =
+                ld_nc_v4(vc + lane * 8);
+        } else if (tid < 96) {
+            if (room)
+                reinterpret_cast<uint4*>(a.s.pend_k + ((size_t)bg * a.s.P + pend_fill) * kHeadDim)[lane] =
+                    ld_nc_v4(a.cand_k + (size_t)bg * kHeadDim + lane * 8);
+        } else if (tid < 128) {
+            if (room)
+                reinterpret_cast<uint4*>(a.s.pend_v + ((size_t)bg * a.s.P + pend_fill) * kHeadDim)[lane] =
+                    ld_nc_v4(a.cand_v + (size_t)bg * kHeadDim + lane * 8);
+        }
+    }
+    if (tid == 128) {
         if (room) a.s.pend_score[(size_t)bg * a.s.P + pend_fill] = a.cand_score[bg];
         else atomicOr(a.s.status, (unsigned)RMA_STATUS_PENDING_OVERFLOW);
         int32_t* c = a.s.counters + bg * 4;
@@ -546,19 +915,87 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
 }
 
+// Every row of every array of one layer, one warp per row: BF16 -> E4M3 codes + exponent.
+__global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ LayerView d,
+                                                       const __grid_constant__ LayerView s) {
+    const int lane = threadIdx.x & 31;
+    const long long nbg = (long long)s.B * s.G;
+    const long long n_ring = nbg * s.R, n_bank = nbg * s.A, n_pend = nbg * s.P;
+    const long long total = 2 * (n_ring + n_bank + n_pend);
+    for (long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); w < total; w += (long long)gridDim.x * 8) {
+        long long r = w;
+        const uint16_t* src;
+        uint8_t* dst;
+        int8_t* dexp;
+        if (r < 2 * n_ring) {
+            const bool v = r >= n_ring;
+            const long long idx = v ? r - n_ring : r;
+            src = (v ? s.ring_v : s.ring_k) + idx * kHeadDim;
+            dst = reinterpret_cast<uint8_t*>(v ? d.ring_v : d.ring_k) + idx * kHeadDim;
+            dexp = (v ? d.ring_ve : d.ring_ke) + (idx / s.R) * d.RE + idx % s.R;
+        } else if ((r -= 2 * n_ring) < 2 * n_bank) {
+            const bool v = r >= n_bank;
+            const long long idx = v ? r - n_bank : r;
+            src = (v ? s.bank_v : s.bank_k) + idx * kHeadDim;
+            dst = reinterpret_cast<uint8_t*>(v ? d.bank_v : d.bank_k) + idx * kHeadDim;
+            dexp = (v ? d.bank_ve : d.bank_ke) + (idx / s.A) * d.AE + idx % s.A;
+        } else {
+            r -= 2 * n_bank;
+            const bool v = r >= n_pend;
+            const long long idx = v ? r - n_pend : r;
+            src = (v ? s.pend_v : s.pend_k) + idx * kHeadDim;
+            dst = reinterpret_cast<uint8_t*>(v ? d.pend_v : d.pend_k) + idx * kHeadDim;
+            dexp = (v ? d.pend_ve : d.pend_ke) + (idx / s.P) * d.PE + idx % s.P;
+        }
+        quantize_row_warp(src, dst, dexp, lane);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-    static SmemLimit limit(reinterpret_cast<const void*>(decode_kernel));
-    const cudaError_t e = limit.ensure(kSmemBytes);
-    if (e != cudaSuccess) return e;
     if (a.ring_splits + a.bank_splits > kMaxSplits) return cudaErrorInvalidValue;
-    dim3 grid(a.ring_splits + a.bank_splits, a.s.G, a.s.B);
-    decode_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);
-    return cudaGetLastError();
+    // launched with programmatic stream serialisation: the kernel's griddepcontrol.wait keeps it
+    // correct after any kernel, and after a decode it overlaps that kernel's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.ring_splits + a.bank_splits, a.s.G, a.s.B);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (a.s.fp8) {
+        static SmemLimit limit(reinterpret_cast<const void*>(decode_kernel<true>));
+        const cudaError_t e = limit.ensure(Smem<true>::kBytes);
+        if (e != cudaSuccess) return e;
+        cfg.dynamicSmemBytes = Smem<true>::kBytes;
+        return cudaLaunchKernelEx(&cfg, decode_kernel<true>, a);
+    }
+    static SmemLimit limit(reinterpret_cast<const void*>(decode_kernel<false>));
+    const cudaError_t e = limit.ensure(Smem<false>::kBytes);
+    if (e != cudaSuccess) return e;
+    cfg.dynamicSmemBytes = Smem<false>::kBytes;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<false>, a);
 }
 
-int decode_max_splits() { return kMaxSplits; }
+cudaError_t launch_quantize_layer(const LayerView& dst, const LayerView& src, cudaStream_t stream) {
+    const long long rows = 2LL * src.B * src.G * ((long long)src.R + src.A + src.P);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long blocks = std::min<long long>((rows + 7) / 8, (long long)sms * 8);
+    quantize_kernel<<<(unsigned)blocks, 256, 0, stream>>>(dst, src);
+    cudaError_t e = cudaGetLastError();
+    const size_t nbg = (size_t)src.B * src.G;
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dst.bank_score, src.bank_score, nbg * src.A * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dst.pend_score, src.pend_score, nbg * src.P * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dst.counters, src.counters, nbg * 16, cudaMemcpyDeviceToDevice, stream);
+    return e;
+}
 
 // ---------------------------------------------------------------------------
 // Built-in decode scratch, for callers that cannot allocate device memory.

@@ -54,6 +54,7 @@ struct State {
     int ring_splits_override;
     int bank_splits_override;
     int sm_count;
+    int decode_overlap;    // rma_set_decode_overlap
 };
 
 // Per-call view of one layer of the state, with device pointers already
@@ -71,7 +72,21 @@ struct LayerView {
     uint32_t* tickets;     // [B][G]
     uint32_t* status;
     int B, G, R, A, P;
+    // FP8 storage (fp8 != 0): the K/V pointers above hold u8 E4M3 codes with the same shapes
+    // (reinterpret them as bytes), and each row's scale exponent lives in these arrays,
+    // [B][G][RE] etc., RE / AE / PE = R / A / P rounded up to 16 (null in a BF16 state)
+    int fp8;
+    int8_t* ring_ke;
+    int8_t* ring_ve;
+    int8_t* bank_ke;
+    int8_t* bank_ve;
+    int8_t* pend_ke;
+    int8_t* pend_ve;
+    int RE, AE, PE;
 };
+
+// Bytes of one stored K or V row.
+__host__ __device__ __forceinline__ int row_bytes(const LayerView& s) { return s.fp8 ? kHeadDim : kRowBytes; }
 
 struct DecodeArgs {
     LayerView s;
@@ -88,6 +103,7 @@ struct DecodeArgs {
     int ring_splits, bank_splits;
     int ring_chunk, bank_chunk; // rows per split (multiples of 16)
     float qscale;               // softmax_scale * log2(e)
+    int early;                  // 1: stream the ring and bank before waiting on the previous launch
 };
 
 struct PrefillArgs {
@@ -121,6 +137,8 @@ cudaError_t launch_admit(const LayerView& s, int force, cudaStream_t stream);
 // Longest prefill block (tokens per sequence) one rma_prefill_block call takes.
 constexpr int kMaxPrefillTokens = 256;
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+// Quantise every row of `src` (BF16) into `dst` (FP8), one layer at a time; scores and counters copied.
+cudaError_t launch_quantize_layer(const LayerView& dst, const LayerView& src, cudaStream_t stream);
 size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok);
 
 }  // namespace rma

@@ -104,7 +104,7 @@ struct Tmaps {
 
 enum Bar {
     kQReady = 0,                // even CTA: 16 arrivals (8 warps x 2 CTAs)
-    kFull = 1,                  // [5] even CTA: own loads (tx) + the odd CTA's signal; odd CTA: own loads
+    kFull = 1,                  // [5] both: this CTA's own loads of the stage landed (tx bytes)
     kEmpty = 6,                 // [5] both: the MMA commit after P V of the chunk in that stage (the stage,
                                 //     that P buffer and O are free to reuse)
     kSFull = 11,                // [2] both, one per softmax group: MMA commit after Q K^T
@@ -112,7 +112,11 @@ enum Bar {
     kSFree = 15,                // [2] even CTA, per group: S has been read, 8 arrivals
     kXfer = 17,                 // both: the other CTA's half-result rows have landed (tx bytes)
     kOFinal = 18,               // both: MMA commit after the last P V (one phase)
-    kNumBars = 19
+    kPeer = 19,                 // [5] even CTA: the odd CTA's half of the stage landed and its stale V rows
+                                //     are cleared (one remote arrival)
+    kDrain = 24,                // both: one commit from each of the even CTA's three MMA-issuing warps after
+                                //     its last MMA: every tensor-core operation of the pair has completed
+    kNumBars = 25
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -179,8 +183,9 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         ptx::mbar_init(&bars[kQReady], 16);
         for (int i = 0; i < kStages; ++i) {
-            ptx::mbar_init(&bars[kFull + i], pr == 0 ? 2 : 1);
+            ptx::mbar_init(&bars[kFull + i], 1);
             ptx::mbar_init(&bars[kEmpty + i], 1);
+            ptx::mbar_init(&bars[kPeer + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars[kSFull + i], 1);
@@ -189,6 +194,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_init(&bars[kXfer], 1);
         ptx::mbar_init(&bars[kOFinal], 1);
+        ptx::mbar_init(&bars[kDrain], 3);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -229,11 +235,13 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         if (warp == kWarpTma) {
             // ---------------- TMA producer: this CTA's half of every chunk ----------------
             const int zreg = b * G + g;
+            int issued = 0;
             for (int j = 0; j < nchunks; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages &&
                     !ptx::mbar_wait_warp(&bars[kEmpty + st], ((j / kStages) - 1) & 1, abort_flag, S.status))
                     break;
+                issued = j + 1;
                 if (lane == 0) {
                     const CUtensorMap* mk;
                     const CUtensorMap* mv;
@@ -260,13 +268,19 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
+            // Drain, normal or abandoned: this CTA's loads of the last stages have landed (earlier
+            // stages were consumed before their reuse), and every MMA of the pair has completed.
+            for (int jj = max(0, issued - kStages); jj < issued; ++jj)
+                ptx::mbar_wait_drain(&bars[kFull + jj % kStages], (jj / kStages) & 1, S.status);
+            ptx::mbar_wait_drain(&bars[kDrain], 0, S.status);
+            __syncwarp();
         } else if (warp == kWarpQK && pr == 1) {
             // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
             for (int j = 0; j < nchunks; ++j) {
                 const int st = j % kStages;
                 if (!ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
                 clear_stale_v(j, st);
-                if (lane == 0) ptx::mbar_arrive_at(&bars[kFull + st], leader, rank);
+                if (lane == 0) ptx::mbar_arrive_at(&bars[kPeer + st], leader, rank);
                 __syncwarp();
             }
             for (int jj = max(0, nchunks - kStages); jj < nchunks; ++jj)
@@ -287,6 +301,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 const int st = j % kStages;
                 ok = ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status);
                 if (!ok) break;
+                ok = ptx::mbar_wait_warp(&bars[kPeer + st], (j / kStages) & 1, abort_flag, S.status);
+                if (!ok) break;
                 clear_stale_v(j, st);
                 ptx::tc_fence_after();
                 if (lane == 0) {
@@ -302,6 +318,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
+            if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
+            __syncwarp();
         } else if (warp == kWarpPV && pr == 0) {
             // ---------------- even CTA: P V issuer ----------------
             // P V of chunk j needs P (which the softmax writes only after reading S of chunk j,
@@ -332,6 +350,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             for (int jj = max(0, nchunks - kStages); ok && jj < nchunks; ++jj)
                 if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
                     break;
+            if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
+            __syncwarp();
         } else if (warp < 8) {
             // ---------------- softmax: thread = (row, half) ----------------
             const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
@@ -579,11 +599,9 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------- tail ----------------
     // The local CTA of this tile combines rows [0, 64), the anchor CTA rows [64, 128): each first
     // pushes the 64 rows the other one needs into that CTA's free stage area [128 KiB, 192 KiB).
-    // After a bounded wait ran out (this CTA abandoned its tile), the copies and tensor-core operations
-    // it had already issued are given ~2 ms to land before the stage area is reused and the CTA exits.
-    if (*abort_flag) {
-        for (int i = 0; i < 2000; ++i) __nanosleep(1000);
-    }
+    // The cluster barrier below follows the producer warp's drain: this CTA's loads have landed and
+    // every tensor-core operation of its pair has completed, also after a wait ran out and the CTA
+    // abandoned its tile, so tensor memory may be freed and the stage area reused.
     __syncwarp();
     ptx::tc_fence_before();
     ptx::cluster_sync();   // all four CTAs have their rows in shared memory; all tensor memory reads done
@@ -602,7 +620,9 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (warp < 8) {
         // one row per warp at a time: lane L makes output dims [8 L, 8 L + 8) (16 contiguous bytes)
-        const bool got = ptx::mbar_wait_warp(&bars[kXfer], 0, abort_flag, S.status);
+        // the partner's copy always comes: wait for it even after an abort, so that it has landed
+        // before this CTA exits
+        const bool got = ptx::mbar_wait_drain(&bars[kXfer], 0, S.status);
 #pragma unroll 2
         for (int rr = 0; rr < 8; ++rr) {
             const int lrow = 8 * warp + rr, crow = 64 * phase + lrow;

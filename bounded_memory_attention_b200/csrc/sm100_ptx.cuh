@@ -65,6 +65,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// A bounded wait that goes on after the CTA has abandoned its tile: it lets operations already
+// issued (TMA loads, tensor-core work, incoming copies) land before their memory is reused or
+// freed.  False, with RMA_STATUS_TIMEOUT set, if the time limit ran out.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(status, (unsigned)RMA_STATUS_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
 // The same wait executed by every lane of a warp, with one verdict for the warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                uint32_t* status) {

@@ -79,9 +79,30 @@ extern "C" {
  * a fault in the library, never an input condition. */
 #define RMA_STATUS_TIMEOUT                  16u
 
+/* Storage of the ring, bank and pending K/V rows (rma_config.kv_format). */
+#define RMA_KV_BF16      0   /* BF16 values, the pages' storage */
+#define RMA_KV_FP8_E4M3  1   /* E4M3 codes with one power-of-two scale per stored row (see below) */
+
 /* Dimensions.  The library implements q_per_group == 4 and head_dim == 256
  * (RMA_ERR_UNSUPPORTED otherwise), any n_groups >= 1, ring_slots in
- * [1, 1<<20], bank_slots >= 1, pend_slots >= 1, bank_slots + pend_slots <= 4096. */
+ * [1, 1<<20], bank_slots >= 1, pend_slots >= 1, bank_slots + pend_slots <= 4096.
+ *
+ * kv_format RMA_KV_FP8_E4M3 halves the K/V bytes ([PRIM] packages paragraph
+ * and [SITE] downloads list: FP8 packages validated for text inference; the
+ * pages do not say how K/V would be stored in FP8, so this storage is the
+ * library's own).  Each stored row (one position's K, or its V, for one KV
+ * group) holds head_dim E4M3 codes (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, no infinities, S.1111.111 = NaN, max 448) and a signed
+ * 8-bit exponent e: the row's values are code * 2^e, e the smallest integer
+ * in [-127, 127] with max|x| <= 448 * 2^e (0 for an all-zero row), the codes
+ * x * 2^-e rounded to nearest, ties to even.  Rows are quantised when written
+ * (the ring write and candidate append of rma_decode_step, and
+ * rma_state_quantize); the admit copies codes, exponents and scores
+ * unchanged; attention reads the stored values, and the current token is
+ * attended as passed in (BF16).  K/V inputs must be finite.  An FP8 state
+ * takes rma_decode_step, rma_decode_step_noalloc, rma_admit and
+ * rma_state_quantize; rma_prefill_block returns RMA_ERR_UNSUPPORTED on it
+ * (prefill a BF16 state, then quantise it). */
 typedef struct rma_config {
     int32_t batch;          /* independent sequences */
     int32_t n_layers;       /* RMA layers (8 in the pages' model) */
@@ -92,6 +113,7 @@ typedef struct rma_config {
     int32_t bank_slots;     /* A (1024) */
     int32_t pend_slots;     /* P (256) */
     float   softmax_scale;  /* 1/sqrt(head_dim) = 1/16 */
+    int32_t kv_format;      /* RMA_KV_BF16 (0) or RMA_KV_FP8_E4M3 (1) */
 } rma_config;
 
 /* Byte offsets, from the start of the caller's state buffer, of each array.
@@ -104,12 +126,19 @@ typedef struct rma_config {
  *   counters              i32   [n_layers][batch][n_groups][4] = {pos, bank_fill, pend_fill, 0}
  *   tickets               u32   [n_layers][batch][n_groups]  (library-internal, zero between calls)
  *   status                u32   one word (RMA_STATUS_* bits)
+ * In an RMA_KV_FP8_E4M3 state the six K/V arrays hold u8 E4M3 codes (same
+ * shapes), and six more arrays hold the rows' scale exponents:
+ *   ring_k_exp, ring_v_exp  i8  [n_layers][batch][n_groups][ring_slots rounded up to 16]
+ *   bank_k_exp, bank_v_exp  i8  [n_layers][batch][n_groups][bank_slots rounded up to 16]
+ *   pend_k_exp, pend_v_exp  i8  [n_layers][batch][n_groups][pend_slots rounded up to 16]
+ * (entries past the slot count are padding); in a BF16 state their offsets are 0.
  * A caller may write the slot arrays and counters directly (to restore a
  * checkpoint or set up a test) while no call is in flight. */
 typedef struct rma_layout {
     uint64_t total_bytes;
     uint64_t ring_k, ring_v, bank_k, bank_v, bank_score;
     uint64_t pend_k, pend_v, pend_score, counters, tickets, status;
+    uint64_t ring_k_exp, ring_v_exp, bank_k_exp, bank_v_exp, pend_k_exp, pend_v_exp;
 } rma_layout;
 
 typedef struct rma_state rma_state;   /* opaque host handle; the device memory is the caller's */
@@ -145,6 +174,23 @@ RMA_API int rma_workspace_bytes(const rma_state* st, int n_tok, size_t* out);
  * (chosen from batch size and SM count).  Affects speed only, not results
  * beyond FP32 summation order. */
 RMA_API int rma_set_decode_splits(rma_state* st, int ring_splits, int bank_splits);
+
+/* Let a decode call start loading its layer's ring and bank while the
+ * previous kernel on the same stream is still finishing (0: off, the default;
+ * 1: on).  Every decode launch may begin before the previous kernel in its
+ * stream ends (programmatic dependent launch), but by default it touches no
+ * global memory until that kernel has completed, which only hides the launch.
+ * With overlap on, the counters are read and the first ring and bank tiles
+ * requested before that point when the previous kernel is a decode call of
+ * this library on another layer of this state (or on another state); the
+ * library tracks this per stream (and per stream capture) and waits first
+ * otherwise.  Inputs and the workspace are always read after the wait, and a
+ * launch never overlaps more than the one before it.  The caller's side of
+ * the contract: while overlap is on, no kernel other than this library's
+ * writes the state between two decode calls on a stream (restoring a
+ * checkpoint with cudaMemcpy is fine; with a kernel of one's own, synchronise
+ * the stream first).  Affects speed only. */
+RMA_API int rma_set_decode_overlap(rma_state* st, int enable);
 
 /* One decode token for every sequence at RMA layer `layer`
  * ([PRIM] operations list, items 1-3; [CARD] "How Rock Memory Anchors work"):
@@ -246,6 +292,13 @@ RMA_API int rma_prefill_block(rma_state* st, int layer, int n_tok,
                       const uint16_t* cand_k, const uint16_t* cand_v, const float* cand_score,
                       const float* w_g, const float* b_g, uint16_t* out,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* Quantise every row of the BF16 state `src` into the RMA_KV_FP8_E4M3 state
+ * `dst` (same dimensions), as rma_config's kv_format describes, and copy the
+ * scores and counters: the way to decode in FP8 after a BF16 prefill.  Every
+ * slot is converted, filled or not.  Both states stay the caller's; they must
+ * not overlap.  RMA_ERR_INVALID_ARG if the formats or dimensions do not match. */
+RMA_API int rma_state_quantize(rma_state* dst, const rma_state* src, void* stream);
 
 /* Wait for `stream`, then read the device status word into *flags and clear it. */
 RMA_API int rma_get_status(rma_state* st, void* stream, uint32_t* flags);

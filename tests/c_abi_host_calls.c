@@ -36,6 +36,14 @@ int main(void) {
     CHECK(two > one && two < 2 * one + 4096);
     cfg.batch = 2;
 
+    /* FP8 storage: one byte per K/V element plus an exponent per row, about half the bytes */
+    cfg.kv_format = RMA_KV_FP8_E4M3;
+    const size_t fp8 = rma_state_bytes(&cfg);
+    CHECK(fp8 > one / 2 && fp8 < one / 2 + one / 50);
+    cfg.kv_format = 7;
+    CHECK(rma_state_bytes(&cfg) == 0);
+    cfg.kv_format = RMA_KV_BF16;
+
     /* an invalid configuration is refused with size 0 and a reason */
     cfg.head_dim = 128;
     CHECK(rma_state_bytes(&cfg) == 0);

@@ -45,13 +45,31 @@ def test_state_size_has_no_sequence_length_input():
     import bounded_memory_attention_b200 as rma
     assert {f for f in rma.Config.__dataclass_fields__} == {
         "batch", "n_layers", "n_groups", "q_per_group", "head_dim", "ring_slots", "bank_slots",
-        "pend_slots", "softmax_scale"}
+        "pend_slots", "softmax_scale", "kv_format"}
+
+
+def test_fp8_state_bytes_are_the_sum_of_codes_exponents_scores_and_counters():
+    """An FP8 state: one byte per K/V element, one exponent byte per row (slots padded to 16),
+    the same scores and counters; per sequence about half the BF16 state."""
+    import bounded_memory_attention_b200 as rma
+    cfg = rma.Config(batch=512, n_layers=8, kv_format=rma.KV_FP8_E4M3)
+    rows = 512 * 8 * 4 * (1023 + 1024 + 256)
+    kv = 2 * rows * 256
+    exps = 2 * 512 * 8 * 4 * (1024 + 1024 + 256)
+    scores = 512 * 8 * 4 * (1024 + 256) * 4
+    counters = 512 * 8 * 4 * (16 + 4) + 4
+    n = rma.state_bytes(cfg)
+    assert kv + exps + scores + counters <= n <= kv + exps + scores + counters + 17 * 256
+    one_bf16 = rma.state_bytes(rma.Config(batch=1, n_layers=8))
+    one_fp8 = rma.state_bytes(rma.Config(batch=1, n_layers=8, kv_format=rma.KV_FP8_E4M3))
+    assert 0.5 < one_fp8 / one_bf16 < 0.51
 
 
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 128, "RMA_ERR_UNSUPPORTED"), ("q_per_group", 8, "RMA_ERR_UNSUPPORTED"),
     ("batch", 0, "RMA_ERR_INVALID_ARG"), ("ring_slots", 0, "RMA_ERR_INVALID_ARG"),
-    ("softmax_scale", float("nan"), "RMA_ERR_INVALID_ARG"), ("bank_slots", 4000, "RMA_ERR_UNSUPPORTED")])
+    ("softmax_scale", float("nan"), "RMA_ERR_INVALID_ARG"), ("bank_slots", 4000, "RMA_ERR_UNSUPPORTED"),
+    ("kv_format", 2, "RMA_ERR_INVALID_ARG")])
 def test_bad_configs_are_rejected_on_the_host(field, value, code):
     import bounded_memory_attention_b200 as rma
     cfg = rma.Config(**{field: value})

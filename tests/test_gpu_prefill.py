@@ -243,7 +243,8 @@ def test_prefill_block_length_checks():
     rma = lib()
     cfg = rma.Config(batch=1, n_layers=1, ring_slots=100)
     st = rma.State(cfg)
-    assert st.workspace_bytes(1) >= st.workspace_bytes(256) == st.workspace_bytes(100) > 0
+    # a block's workspace never shrinks with its length; a decode step's (n_tok = 1) is positive
+    assert st.workspace_bytes(256) >= st.workspace_bytes(100) > 0 and st.workspace_bytes(1) > 0
     for n, code in ((0, "RMA_ERR_INVALID_ARG"), (257, "RMA_ERR_UNSUPPORTED")):
         with pytest.raises(rma.RmaError) as e:
             st.workspace_bytes(n)
