@@ -87,3 +87,9 @@ def test_null_and_layer_errors_without_a_gpu():
     assert rma.lib.rma_decode_step(None, 0, *([None] * 10), 0, None) == -1
     assert rma.lib.rma_strerror(-3) == b"buffer too small"
     assert rma.lib.rma_strerror(0) == b"ok"
+
+
+def test_setters_reject_null_states_without_a_gpu():
+    import bounded_memory_attention_b200 as rma
+    assert rma.lib.rma_set_decode_overlap(None, 1) == -1
+    assert rma.lib.rma_set_decode_splits(None, 1, 1) == -1
