@@ -9,7 +9,8 @@ order; a tcgen05 commit arrives once every earlier MMA of its issuing thread is 
 
 What it checks, over many random schedules:
   * every parity wait is sound: it is made while its barrier has completed P or P + 1 phases (a
-    barrier two phases ahead would let a parity wait pass on the wrong phase);
+    barrier two phases ahead would let a parity wait pass on the wrong phase, and one whose phase
+    P - 1 is still open would let it pass at once);
   * nothing deadlocks (an abort-aware wait that can never complete is timed out, as the kernel's
     bounded wait would, and its CTA abandons its tile; a drain wait that can never complete is an
     error);
@@ -311,4 +312,10 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
             live.remove(p)
             state[p] = None
             continue
+        nw = state[p]
+        if nw is not None and nw[0] == "wait" and nw[2].done < nw[3] and not (abort[nw[1]] and not nw[4]):
+            # the phase before the awaited one is still open: its parity differs from the awaited
+            # phase's, so the hardware's parity wait would pass at once
+            raise Hazard(f"{p[0]}@{p[1]} waits phase {nw[3]} of {nw[2].name}, which has completed only "
+                         f"{nw[2].done}")
     return steps

@@ -61,3 +61,23 @@ def test_a_parity_wait_two_phases_behind_is_caught():
         except ns["Hazard"]:
             caught += 1
     assert caught > 0
+
+
+def test_a_parity_wait_on_a_phase_not_yet_open_is_caught():
+    """A planted protocol mistake: the P V issuer waits on the P buffer's next phase (the phase
+    before it still open, so the hardware's parity wait would pass at once and P V would read a P
+    not yet written)."""
+    src = open(model.__file__).read()
+    bad = src.replace('ok = yield wait(E, bar[E]["PFull"][j & 1], j >> 1)',
+                      'ok = yield wait(E, bar[E]["PFull"][j & 1], (j >> 1) + 1)')
+    assert bad != src
+    ns = {}
+    exec(compile(bad, "planted_model", "exec"), ns)
+    caught = 0
+    for seed in range(50):
+        try:
+            ns["run"](9, seed)
+        except ns["Hazard"] as e:
+            assert "completed only" in str(e)
+            caught += 1
+    assert caught > 0
