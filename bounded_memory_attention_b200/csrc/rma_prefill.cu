@@ -10,51 +10,63 @@
 // Then the block's K/V go into the ring, its candidates into pending, and
 // the admit runs forced.
 //
-// One launch.  A CTA owns 128 query rows (32 tokens x the group's 4 query
-// heads, which share every key) and one phase: the local window (phase 0) or
-// the bank (phase 1).  Four CTAs form a thread-block cluster:
-//   rank 0: tile 2p, local     rank 1: tile 2p+1, local
-//   rank 2: tile 2p, anchor    rank 3: tile 2p+1, anchor
-// A block may hold any n from 1 to 256 tokens: the grid covers ceil(n / 64)
-// pairs of tiles, rows past the last token repeat its query and are not
-// stored, and keys past it are masked (their V rows cleared).
-// Ranks (0,1) and (2,3) are CTA pairs for the 2-SM tensor-core MMA
-// (tcgen05 cta_group::2, M = 256): both tiles of a pair read exactly the same
-// keys, so each CTA loads only half of every 64-key K/V chunk (K rows split
-// by key, V split by dimension), which halves the K/V bytes per FLOP.
-//   * tensor memory (512 columns, the pair allocates together): O [0,256)
-//     FP32, S double buffer [256,320) and [320,384) (chunk j in S_(j & 1)),
-//     Q [384,512) packed BF16 (Q K^T takes A from tensor memory); shared
-//     memory holds a five-stage ring of K/V half-chunks and one BF16 P buffer
-//     per softmax group (the UMMA K-major layout, 128-byte swizzle);
-//   * warp 8 of each CTA loads its half of each chunk with TMA (128B swizzle);
-//   * in the even CTA, warps 9 and 11 issue S = Q K^T (N 64, K 256) for even
-//     and odd chunks and warp 10 issues O += P V (N 256, K 64, P and V from
-//     shared memory, V an MN-major operand), committing to the barriers of both
-//     CTAs; the tensor pipe queues few instructions, and three issuers keep it
-//     fed while any one waits.  Warp 9 of the odd CTA checks its half landed,
-//     clears stale V rows and signals the even CTA;
-//   * warps 0-7 of each CTA are the softmax for its own rows: two
-//     warpgroups that take alternate chunks, each thread a whole 64-key row;
-//     they load Q into tensor memory (and compute the gate), read S, release
-//     its columns for Q K^T of chunk j + 2, mask by position (32-key halves
-//     that are all visible skip the per-key test), hand the reference max from
-//     chunk to chunk through shared memory (moving it only when a chunk's max
-//     exceeds it by more than 2^8, then rescaling O), write P to shared memory,
-//     keep one row sum per group and finally normalise O.
-// Tail: every CTA writes its normalised rows into its own shared memory and
-// pushes the 64 rows the other CTA of its tile (local <-> anchor) combines into
-// that CTA's free stage area with one bulk copy (no multicast); each combines
-// its half: out = local + gate * anchor in FP32, rounded once to BF16.  Each CTA
-// appends its share of the candidates to pending; local pairs write the block's
-// K/V into the ring as soon as every earlier pair has finished reading it; the
-// last CTA of the (sequence, group) runs the forced admit.  No load is
-// multicast: every CTA reads its own data.
+// Three launches.
+//
+// 1. prefill_attn_kernel, persistent: one cluster of 2 CTAs per pair of SMs,
+//    each cluster looping over work items.  An item is one (sequence, group,
+//    pair of tiles, phase): a tile is 32 tokens x the group's 4 query heads =
+//    128 query rows, the two tiles of a pair are the two CTAs of a tcgen05
+//    cta_group::2 MMA pair (M = 256; both read exactly the same keys, so each
+//    CTA loads only half of every 64-key K/V chunk), and the phase is the local
+//    window (ring + block, causal) or the bank.  Items run in (sequence,
+//    group)-major order, a group's local items before its anchor items.  Per
+//    CTA and item:
+//      * tensor memory (512 columns, allocated once): O [0,256) FP32, S double
+//        buffer [256,320) / [320,384), Q [384,512) packed BF16 (Q K^T takes A
+//        from tensor memory); shared memory holds a five-stage ring of K/V
+//        half-chunks (128-byte swizzle) and one BF16 P buffer per softmax group;
+//      * warp 8 loads this CTA's half of each chunk with TMA; in the even CTA
+//        warps 9 and 11 issue S = Q K^T for even and odd chunks and warp 10
+//        issues O += P V (the tensor pipe queues few instructions, so three
+//        issuers keep it fed); warp 9 of the odd CTA checks its half landed,
+//        clears stale V rows and signals the even CTA;
+//      * warps 0-7 are the softmax: two groups taking alternate chunks, each
+//        thread a whole 64-key row, the reference max handed from chunk to chunk
+//        through shared memory (moved only when a chunk's max exceeds it by more
+//        than 2^8, O rescaled then).  At the end of the item they write the
+//        normalised rows (FP32) to the workspace, 32 columns at a time through
+//        their P buffer and a TMA store, and go on to the next item, whose first
+//        K/V chunks are already loaded and whose query rows the TMA warp has
+//        asked L2 for; the P V issuer starts that item's P V once both CTAs have
+//        read O.
+//    Every barrier phase follows a chunk counter (or a counter of the items
+//    that have chunks) running on across items.  A group's counters are
+//    constant while any of its items runs: the second launch writes them only
+//    after every item of the group has finished.
+// 2. prefill_commit_kernel, launched with programmatic stream serialisation
+//    so that its CTAs are scheduled as soon as SMs free up: per (sequence,
+//    group), slice CTAs append their tokens' candidates to pending and compute
+//    the gate tanh(q . w_g + b_g) of their rows at once (neither is read by the
+//    first launch), wait until every item of their group has stored its rows
+//    (the items count themselves in the high half of the group's ticket word
+//    once their TMA stores have completed; items run in group-major order, so
+//    most groups are done well before the last), then combine out = local +
+//    gate * anchor in FP32, rounded once to BF16, and write the block's K/V into
+//    the ring (every read of the group's ring is done); one CTA runs the forced
+//    admit's competition (scores only, no wait) and leaves the list of admitted
+//    candidates and their bank slots in the workspace; the last CTA of the group
+//    to arrive writes the counters.
+// 3. prefill_admit_copy_kernel, launched the same way after the commit, which
+//    it waits for with griddepcontrol.wait (and so for every item of every
+//    group): the admitted rows (pending rows, or the block's own candidates from
+//    the inputs) into their bank slots.
+// No load is multicast: every CTA reads its own data.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "rma_admit_impl.cuh"
@@ -78,46 +90,84 @@ constexpr int kSmemP = kStages * kStageBytes;         // 160 KiB: P of the two s
 constexpr int kPBytes = 128 * 128;                    // 128 rows x 64 keys (BF16), 128-byte swizzle
 constexpr int kSmemBar = kSmemP + 2 * kPBytes;        // 192 KiB
 // softmax exchange (floats): the reference max handed between the groups [128] at 0, each
-// group's final reference max [2][128] at 128 and row sum [2][128] at 512, the gate [128] at 768
-// (first the two halves' partial dot products [2][128], then the gate itself in the first)
+// group's final reference max [2][128] at 128 and row sum [2][128] at 512
 constexpr int kSmemXch = kSmemBar + 512;
-constexpr int kSmemW = kSmemXch + 4096;               // w_g rows of the group's 4 heads (FP32)
-constexpr int kSmemBytes = kSmemW + 4096 + 1024;      // + 1 KiB for alignment
-constexpr int kXchEndM = 128, kXchEndL = 512, kXchGate = 768;
+constexpr int kSmemBytes = kSmemXch + 4096 + 1024;    // + 1 KiB for alignment
+constexpr int kXchEndM = 128, kXchEndL = 512;
 constexpr int kSoftmaxThreads = 256;                  // warps 0-7
-// warp 8: TMA producer; warps 9 and 11: Q K^T issuers for even and odd chunks (even CTA;
-// in the odd CTA warp 9 is the stale-row cleaner); warp 10: P V issuer (even CTA).  The
-// tensor pipe queues few instructions, so it idles whenever its only issuer waits on a
-// barrier; three issuing warps keep it fed while any one of them waits.
 constexpr int kWarpTma = 8, kWarpQK = 9, kWarpPV = 10, kWarpQK2 = 11;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
-constexpr int kTilesPerCluster = 2;
+constexpr int kCommitThreads = 256;
+constexpr int kCommitSlices = 16;                     // slice CTAs per (sequence, group) in the commit
+constexpr int kCommitUnroll = 4;                      // combine elements a thread loads before it stores
 
-static_assert(kSmemBar >= kRows * 1024, "the result rows reuse the K/V stages");
-static_assert(kSmemBar >= (int)admit_scratch_bytes(1, 4095), "the tail's admit reuses the K/V stages");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct Tmaps {
     CUtensorMap k, v, ring_k, ring_v, bank_k, bank_v;   // K maps: 32-row boxes; V maps: 64-row boxes
+    CUtensorMap ws;   // FP32 [phase][b][t][head][256], boxes of 32 dims x 4 heads x 32 tokens
 };
 
 enum Bar {
-    kQReady = 0,                // even CTA: 16 arrivals (8 warps x 2 CTAs)
-    kFull = 1,                  // [5] both: this CTA's own loads of the stage landed (tx bytes)
-    kEmpty = 6,                 // [5] both: the MMA commit after P V of the chunk in that stage (the stage,
-                                //     that P buffer and O are free to reuse)
-    kSFull = 11,                // [2] both, one per softmax group: MMA commit after Q K^T
-    kPFull = 13,                // [2] even CTA, per group: P is in shared memory, 8 arrivals (4 warps x 2 CTAs)
-    kSFree = 15,                // [2] even CTA, per group: S has been read, 8 arrivals
-    kXfer = 17,                 // both: the other CTA's half-result rows have landed (tx bytes)
-    kOFinal = 18,               // both: MMA commit after the last P V (one phase)
-    kPeer = 19,                 // [5] even CTA: the odd CTA's half of the stage landed and its stale V rows
-                                //     are cleared (one remote arrival)
-    kDrain = 24,                // both: one commit from each of the even CTA's three MMA-issuing warps after
-                                //     its last MMA: every tensor-core operation of the pair has completed
+    kQReady = 0,      // even CTA, per item with chunks: 16 arrivals (8 softmax warps x 2 CTAs): Q in TMEM
+    kFull = 1,        // [5] both: this CTA's own loads of the stage landed (tx bytes)
+    kEmpty = 6,       // [5] both: MMA commit after P V of the chunk in that stage
+    kSFull = 11,      // [2] both: MMA commit after Q K^T into S buffer jg & 1
+    kPFull = 13,      // [2] even CTA: P of chunk jg in shared memory, 8 arrivals (4 warps x 2 CTAs)
+    kSFree = 15,      // [2] even CTA: S of chunk jg read, 8 arrivals
+    kOFinal = 17,     // both, per item with chunks: MMA commit after the item's last P V
+    kODrained = 18,   // even CTA, per item with chunks: O read by the 8 softmax warps of both CTAs (16)
+    kPeer = 19,       // [5] even CTA: the odd CTA's half of the stage landed, stale V rows cleared
+    kDrain = 24,      // both: one commit from each of the even CTA's three MMA-issuing warps after its last MMA
     kNumBars = 25
 };
+
+// The workspace: normalised local rows and anchor rows, each [B][n][HQ][256] FP32.
+__host__ __device__ __forceinline__ size_t ws_rows_floats(int B, int n, int HQ) {
+    return (size_t)B * n * HQ * kHeadDim;
+}
+// After the rows: per (sequence, group) the admit's list, [n_adm, pend_fill, -, -, src[P], dest[P]]
+// (ints): admitted candidate t (pending slot t if t < pend_fill, else block token t - pend_fill)
+// goes to bank slot dest, in ascending t.
+__host__ __device__ __forceinline__ size_t admit_list_ints(int P) { return 4 + 2 * (size_t)P; }
+__device__ __forceinline__ int* admit_list(float* ws, int B, int n, int HQ, int P, int bg) {
+    return reinterpret_cast<int*>(ws + 2 * ws_rows_floats(B, n, HQ)) + (size_t)bg * admit_list_ints(P);
+}
+
+// One work item: tiles 2p and 2p+1 of (sequence b, group g) in one phase (0 local, 1 bank).
+struct Item {
+    int b, g, bg, p, phase;
+    int s, bank_fill, pend_fill, fill;
+    int n_ring, n_blk, n_bank, nchunks;
+};
+
+// Items in (sequence, group)-major order, the local items of a group before its anchor items, so
+// that groups complete one after another and their commits can start before the launch ends.
+__device__ __forceinline__ Item make_item(const LayerView& S, int it, int npairs) {
+    Item x;
+    x.bg = it / (2 * npairs);
+    const int r = it % (2 * npairs);
+    x.phase = r / npairs;
+    x.p = r % npairs;
+    x.g = x.bg % S.G;
+    x.b = x.bg / S.G;
+    const int32_t* cnt = S.counters + x.bg * 4;
+    x.s = max(cnt[0], 0);
+    x.bank_fill = min(max(cnt[1], 0), S.A);
+    x.pend_fill = min(max(cnt[2], 0), S.P);
+    x.fill = min(x.s, S.R);
+    x.n_ring = x.n_blk = x.n_bank = 0;
+    if (x.phase == 0) {
+        x.n_ring = (x.fill + kChunk - 1) / kChunk;
+        x.n_blk = x.p + 1;                       // tiles 2p and 2p+1 reach block chunk p
+    } else {
+        x.n_bank = (x.bank_fill + kChunk - 1) / kChunk;
+    }
+    x.nchunks = x.n_ring + x.n_blk + x.n_bank;
+    return x;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -130,57 +180,100 @@ __device__ __forceinline__ float fast_ex2(float x) {
     return y;
 }
 
-__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ Tmaps tm, const __grid_constant__ PrefillArgs a, int ntiles) {
+// TMA store of one box of the FP32 workspace from shared memory (bulk-group completion)
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3,
+                                             int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4, %5}], [%6];\n" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(ptx::smem_u32(src))
+        : "memory");
+}
+// Wait until every bulk store this thread committed has completed (its writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// Ask for `bytes` (a multiple of 16) at a 16-byte aligned global address to be brought into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
+// Wait (bounded) until the high half of the group's ticket word reaches `need`; on timeout the
+// status word gets RMA_STATUS_TIMEOUT and the caller goes on (its results are then undefined).
+__device__ __forceinline__ void wait_rows(const LayerView& S, int bg, unsigned need) {
+    if (threadIdx.x == 0) {
+        const long long t0 = clock64();
+        unsigned v;
+        while (true) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(S.tickets + bg) : "memory");
+            if ((v >> 16) >= need) break;
+            if (clock64() - t0 > ptx::kWaitLimitCycles) {
+                atomicOr(S.status, (unsigned)RMA_STATUS_TIMEOUT);
+                break;
+            }
+            __nanosleep(256);
+        }
+    }
+    __syncthreads();
+    __threadfence();
+}
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// number of valid keys of chunk j of item x (rows past it may hold stale bytes)
+__device__ __forceinline__ int chunk_valid(const Item& x, int j, int n) {
+    if (j < x.n_ring) return x.fill - kChunk * j;
+    if (j < x.n_ring + x.n_blk) return n - kChunk * (j - x.n_ring);
+    return x.bank_fill - kChunk * (j - x.n_ring - x.n_blk);
+}
+
+// clear V rows [nvalid, 64) of this CTA's half in stage st so that P = 0 times V stays 0 (one warp)
+__device__ __forceinline__ void clear_stale_v(uint8_t* smem, int nvalid, int st, int lane) {
+    if (nvalid < kChunk) {
+        uint8_t* vst = smem + st * kStageBytes + kKHalfBytes;
+        const int nz = (kChunk - nvalid) * 8;   // 16-byte pieces per slab
+        for (int e = lane; e < 2 * nz; e += 32) {
+            const int slab = e / nz, piece = e % nz;
+            reinterpret_cast<uint4*>(vst + slab * kSlabV + nvalid * 128)[piece] = make_uint4(0, 0, 0, 0);
+        }
+        ptx::fence_proxy_async_smem();
+    }
+    __syncwarp();
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    prefill_attn_kernel(const __grid_constant__ Tmaps tm, const __grid_constant__ PrefillArgs a, int npairs,
+                        int n_items) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const LayerView& S = a.s;
     const uint32_t rank = ptx::cluster_ctarank();
     const int pr = rank & 1;                     // 0: the pair's MMA-issuing CTA
-    const int phase = rank >> 1;
-    const int T = kTilesPerCluster * (blockIdx.x >> 2) + pr;
-    const int g = blockIdx.y, b = blockIdx.z;
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = S.G, HQ = G * kQPerGroup, n = a.n_tok;
-    const int bg = b * G + g;
-    const uint32_t leader = rank & ~1u;
-    const uint16_t pair_mask = (uint16_t)(3u << leader);
+    const uint16_t pair_mask = 3u;
+    const uint32_t leader = 0;
 
-    const int32_t* cnt = S.counters + bg * 4;
-    const int c_pos = cnt[0], c_bank = cnt[1], c_pend = cnt[2];
-    if ((c_pos < 0 || c_bank < 0 || c_bank > S.A || c_pend < 0 || c_pend > S.P) && threadIdx.x == 0 && rank == 0 &&
-        blockIdx.x == 0)
-        atomicOr(S.status, (unsigned)RMA_STATUS_BAD_COUNTERS);   // a corrupted state: clamped below
-    const int s = max(c_pos, 0);
-    const int bank_fill = min(max(c_bank, 0), S.A);
-    const int pend_fill = min(max(c_pend, 0), S.P);
-    const int fill = min(s, S.R);
-
-    // chunks (identical for both CTAs of a pair: tiles 2p and 2p+1 need block chunks 0..p)
-    int n_ring = 0, n_blk = 0, n_bank = 0;
-    if (phase == 0) {
-        n_ring = (fill + kChunk - 1) / kChunk;
-        n_blk = (kTileTok * (T | 1) + kTileTok - 1) / kChunk + 1;
-    } else {
-        n_bank = (bank_fill + kChunk - 1) / kChunk;
-    }
-    const int nchunks = n_ring + n_blk + n_bank;
-    const bool has_work = nchunks > 0;        // uniform over the pair
+    // the commit launch may be scheduled now: it waits for this grid's completion before it reads
+    grid_dep_launch();
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars + 1);
-    int* tail_flag = reinterpret_cast<int*>(bars + kNumBars + 2);
-
-    const int row = 32 * (warp & 3) + lane;   // softmax threads: row of this CTA
-    const int wg = (warp >> 2) & 1;           // and which half of keys / columns
-    const int tok = kTileTok * T + (row >> 2);
-    const int head = g * kQPerGroup + (row & 3);
     float* xch = reinterpret_cast<float*>(smem + kSmemXch);
-    float l = 0.f;
-    uint32_t tmem = 0;
 
     if (tid == 0) {
+        if (cluster == 0 && rank == 0) {
+            // a corrupted state is clamped for indexing (make_item); flag it once
+            for (int bg = 0; bg < S.B * G; ++bg) {
+                const int32_t* c = S.counters + bg * 4;
+                if (c[0] < 0 || c[1] < 0 || c[1] > S.A || c[2] < 0 || c[2] > S.P) {
+                    atomicOr(S.status, (unsigned)RMA_STATUS_BAD_COUNTERS);
+                    break;
+                }
+            }
+        }
         ptx::mbar_init(&bars[kQReady], 16);
         for (int i = 0; i < kStages; ++i) {
             ptx::mbar_init(&bars[kFull + i], 1);
@@ -192,71 +285,57 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars[kPFull + i], 8);
             ptx::mbar_init(&bars[kSFree + i], 8);
         }
-        ptx::mbar_init(&bars[kXfer], 1);
         ptx::mbar_init(&bars[kOFinal], 1);
+        ptx::mbar_init(&bars[kODrained], 16);
         ptx::mbar_init(&bars[kDrain], 3);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (tid < kSoftmaxThreads)   // the gate weights of the group's heads, one float4 per thread
-        reinterpret_cast<float4*>(smem + kSmemW)[tid] =
-            __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)g * kQPerGroup * kHeadDim) + tid);
-    if (has_work && warp == kWarpQK) {
+    if (warp == kWarpQK) {
         ptx::tmem_alloc2(tmem_holder, kTmemCols);
         ptx::tmem_relinquish2();
     }
     ptx::tc_fence_before();
-    ptx::cluster_sync();   // barriers of all four CTAs initialised, tensor memory allocated
+    ptx::cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     ptx::tc_fence_after();
-    if (has_work) tmem = *tmem_holder;
+    const uint32_t tmem = *tmem_holder;
 
-    // number of valid keys of chunk j (rows past it may hold stale bytes)
-    auto chunk_valid = [&](int j) -> int {
-        if (j < n_ring) return fill - kChunk * j;
-        if (j < n_ring + n_blk) return n - kChunk * (j - n_ring);
-        return bank_fill - kChunk * (j - n_ring - n_blk);
-    };
-    // clear V rows [nvalid, 64) of this CTA's half in stage st so that P = 0 times V stays 0
-    auto clear_stale_v = [&](int j, int st) {
-        const int nvalid = chunk_valid(j);
-        if (nvalid < kChunk) {
-            uint8_t* vst = smem + st * kStageBytes + kKHalfBytes;
-            const int nz = (kChunk - nvalid) * 8;   // 16-byte pieces per slab
-            for (int e = lane; e < 2 * nz; e += 32) {
-                const int slab = e / nz, piece = e % nz;
-                reinterpret_cast<uint4*>(vst + slab * kSlabV + nvalid * 128)[piece] = make_uint4(0, 0, 0, 0);
+    if (warp == kWarpTma) {
+        // ---------------- TMA producer: this CTA's half of every chunk of every item ----------------
+        int jg = 0, issued = 0;
+        bool ok = true;
+        for (int it = cluster; ok && it < n_items; it += n_clusters) {
+            const Item x = make_item(S, it, npairs);
+            if (it + n_clusters < n_items) {
+                // the next item's query rows of this CTA into L2 (one token's 4 heads per lane): its
+                // softmax threads load them when that item starts
+                const Item y = make_item(S, it + n_clusters, npairs);
+                const int t = kTileTok * (2 * y.p + pr) + lane;
+                if (t < n) prefetch_l2(a.q + ((size_t)(y.b * n + t) * HQ + y.g * kQPerGroup) * kHeadDim, kQPerGroup * kRowBytes);
             }
-            ptx::fence_proxy_async_smem();
-        }
-        __syncwarp();
-    };
-
-    if (has_work) {
-        if (warp == kWarpTma) {
-            // ---------------- TMA producer: this CTA's half of every chunk ----------------
-            const int zreg = b * G + g;
-            int issued = 0;
-            for (int j = 0; j < nchunks; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages &&
-                    !ptx::mbar_wait_warp(&bars[kEmpty + st], ((j / kStages) - 1) & 1, abort_flag, S.status))
+            for (int j = 0; j < x.nchunks; ++j, ++jg) {
+                const int st = jg % kStages;
+                if (jg >= kStages &&
+                    !ptx::mbar_wait_warp(&bars[kEmpty + st], ((jg / kStages) - 1) & 1, abort_flag, S.status)) {
+                    ok = false;
                     break;
-                issued = j + 1;
+                }
+                issued = jg + 1;
                 if (lane == 0) {
                     const CUtensorMap* mk;
                     const CUtensorMap* mv;
                     int yk, zk, yv, zv;
-                    if (j < n_ring) {
+                    if (j < x.n_ring) {
                         mk = &tm.ring_k; mv = &tm.ring_v;
-                        yk = kChunk * j + kHalfKeys * pr; zk = zreg; yv = kChunk * j; zv = zreg;
-                    } else if (j < n_ring + n_blk) {
-                        const int t0 = b * n + kChunk * (j - n_ring);
+                        yk = kChunk * j + kHalfKeys * pr; zk = x.bg; yv = kChunk * j; zv = x.bg;
+                    } else if (j < x.n_ring + x.n_blk) {
+                        const int t0 = x.b * n + kChunk * (j - x.n_ring);
                         mk = &tm.k; mv = &tm.v;
-                        yk = g; zk = t0 + kHalfKeys * pr; yv = g; zv = t0;
+                        yk = x.g; zk = t0 + kHalfKeys * pr; yv = x.g; zv = t0;
                     } else {
-                        const int a0 = kChunk * (j - n_ring - n_blk);
+                        const int a0 = kChunk * (j - x.n_ring - x.n_blk);
                         mk = &tm.bank_k; mv = &tm.bank_v;
-                        yk = a0 + kHalfKeys * pr; zk = zreg; yv = a0; zv = zreg;
+                        yk = a0 + kHalfKeys * pr; zk = x.bg; yv = a0; zv = x.bg;
                     }
                     uint8_t* stage = smem + st * kStageBytes;
                     ptx::mbar_arrive_expect_tx(&bars[kFull + st], kStageBytes);
@@ -268,72 +347,97 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-            // Drain, normal or abandoned: this CTA's loads of the last stages have landed (earlier
-            // stages were consumed before their reuse), and every MMA of the pair has completed.
-            for (int jj = max(0, issued - kStages); jj < issued; ++jj)
-                ptx::mbar_wait_drain(&bars[kFull + jj % kStages], (jj / kStages) & 1, S.status);
-            ptx::mbar_wait_drain(&bars[kDrain], 0, S.status);
-            __syncwarp();
-        } else if (warp == kWarpQK && pr == 1) {
-            // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
-            for (int j = 0; j < nchunks; ++j) {
-                const int st = j % kStages;
-                if (!ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status)) break;
-                clear_stale_v(j, st);
+        }
+        // Drain, normal or abandoned: this CTA's loads of the last stages have landed (earlier
+        // stages were consumed before their reuse), and every MMA of the pair has completed.
+        for (int jj = max(0, issued - kStages); jj < issued; ++jj)
+            ptx::mbar_wait_drain(&bars[kFull + jj % kStages], (jj / kStages) & 1, S.status);
+        ptx::mbar_wait_drain(&bars[kDrain], 0, S.status);
+        __syncwarp();
+    } else if (warp == kWarpQK && pr == 1) {
+        // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
+        int jg = 0;
+        bool ok = true;
+        for (int it = cluster; ok && it < n_items; it += n_clusters) {
+            const Item x = make_item(S, it, npairs);
+            for (int j = 0; j < x.nchunks; ++j, ++jg) {
+                const int st = jg % kStages;
+                if (!ptx::mbar_wait_warp(&bars[kFull + st], (jg / kStages) & 1, abort_flag, S.status)) {
+                    ok = false;
+                    break;
+                }
+                clear_stale_v(smem, chunk_valid(x, j, n), st, lane);
                 if (lane == 0) ptx::mbar_arrive_at(&bars[kPeer + st], leader, rank);
                 __syncwarp();
             }
-            for (int jj = max(0, nchunks - kStages); jj < nchunks; ++jj)
-                if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
-                    break;
-        } else if (warp == kWarpQK || (warp == kWarpQK2 && pr == 0)) {
-            // ---------------- even CTA: Q K^T issuers (warp 9: even chunks, warp 11: odd) ----------------
-            // S of chunk j lives in columns kColS0 / kColS1 by j & 1 and P in shared memory, so
-            // Q K^T of chunk j + 2 may start as soon as the softmax group has read S of chunk j.
-            constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(2 * kRows, kChunk, false, false);
-            bool ok = ptx::mbar_wait_warp(&bars[kQReady], 0, abort_flag, S.status);
+        }
+        // consume the last stages' empty phases (commits into this CTA's barriers)
+        for (int jj = max(0, jg - kStages); ok && jj < jg; ++jj)
+            if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status)) break;
+    } else if (warp == kWarpQK || (warp == kWarpQK2 && pr == 0)) {
+        // ---------------- even CTA: Q K^T issuers (warp 9: even global chunks, warp 11: odd) ----------------
+        constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(2 * kRows, kChunk, false, false);
+        const int mine = warp == kWarpQK ? 0 : 1;
+        int jg = 0, kw = 0;
+        bool ok = true;
+        for (int it = cluster; ok && it < n_items; it += n_clusters) {
+            const Item x = make_item(S, it, npairs);
+            if (x.nchunks == 0) continue;        // an empty bank: no Q K^T, and its Q is not loaded
+            // Q of this item is in tensor memory (phase kw of kQReady).  Both issuers wait for every
+            // phase, in order, even in an item where one of them has no chunk: a parity wait on a
+            // barrier two phases ahead would pass at once.
+            ok = ptx::mbar_wait_warp(&bars[kQReady], kw & 1, abort_flag, S.status);
+            ++kw;
             ptx::tc_fence_after();
-            for (int j = warp == kWarpQK ? 0 : 1; ok && j < nchunks; j += 2) {
-                if (j >= 2) {
-                    ok = ptx::mbar_wait_warp(&bars[kSFree + (j & 1)], ((j - 2) >> 1) & 1, abort_flag, S.status);
+            for (int j = 0; ok && j < x.nchunks; ++j, ++jg) {
+                if ((jg & 1) != mine) continue;
+                if (jg >= 2) {
+                    ok = ptx::mbar_wait_warp(&bars[kSFree + (jg & 1)], ((jg - 2) >> 1) & 1, abort_flag, S.status);
                     if (!ok) break;
                 }
-                const int st = j % kStages;
-                ok = ptx::mbar_wait_warp(&bars[kFull + st], (j / kStages) & 1, abort_flag, S.status);
+                const int st = jg % kStages;
+                ok = ptx::mbar_wait_warp(&bars[kFull + st], (jg / kStages) & 1, abort_flag, S.status);
                 if (!ok) break;
-                ok = ptx::mbar_wait_warp(&bars[kPeer + st], (j / kStages) & 1, abort_flag, S.status);
+                ok = ptx::mbar_wait_warp(&bars[kPeer + st], (jg / kStages) & 1, abort_flag, S.status);
                 if (!ok) break;
-                clear_stale_v(j, st);
+                clear_stale_v(smem, chunk_valid(x, j, n), st, lane);
                 ptx::tc_fence_after();
                 if (lane == 0) {
                     const uint32_t k_base = ptx::smem_u32(smem + st * kStageBytes);
-                    const uint32_t d = tmem + ((j & 1) ? kColS1 : kColS0);
+                    const uint32_t d = tmem + ((jg & 1) ? kColS1 : kColS0);
                     for (int ks = 0; ks < kHeadDim / 16; ++ks) {
                         // 16 dims = 32 bytes inside the 128-byte swizzle atom of slab ks / 4
                         const uint64_t bd = ptx::smem_desc(k_base + (ks >> 2) * kSlabK + (ks & 3) * 32, 16, 1024,
                                                            ptx::kSwizzle128B);
                         ptx::mma_ts2(d, tmem + kColQ + 8 * ks, bd, idesc_qk, ks > 0 ? 1u : 0u);
                     }
-                    ptx::mma_commit2_mc(&bars[kSFull + (j & 1)], pair_mask);
+                    ptx::mma_commit2_mc(&bars[kSFull + (jg & 1)], pair_mask);
                 }
                 __syncwarp();
             }
-            if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
-            __syncwarp();
-        } else if (warp == kWarpPV && pr == 0) {
-            // ---------------- even CTA: P V issuer ----------------
-            // P V of chunk j needs P (which the softmax writes only after reading S of chunk j,
-            // so Q K^T of chunk j has completed) and V (landed before Q K^T of chunk j was issued).
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(2 * kRows, kHeadDim, false, true);
-            bool ok = true;
-            for (int j = 0; ok && j < nchunks; ++j) {
-                const int st = j % kStages;
-                ok = ptx::mbar_wait_warp(&bars[kPFull + (j & 1)], (j >> 1) & 1, abort_flag, S.status);
+        }
+        if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
+        __syncwarp();
+    } else if (warp == kWarpPV && pr == 0) {
+        // ---------------- even CTA: P V issuer ----------------
+        constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(2 * kRows, kHeadDim, false, true);
+        // kQReady, kOFinal and kODrained count only the items that have chunks (kw of them so far)
+        int jg = 0, kw = 0;
+        bool ok = true;
+        for (int it = cluster; ok && it < n_items; it += n_clusters) {
+            const Item x = make_item(S, it, npairs);
+            if (x.nchunks == 0) continue;
+            // the previous item's O has been read by both CTAs before this item's first P V
+            if (kw >= 1) ok = ptx::mbar_wait_warp(&bars[kODrained], (kw - 1) & 1, abort_flag, S.status);
+            ++kw;
+            for (int j = 0; ok && j < x.nchunks; ++j, ++jg) {
+                const int st = jg % kStages;
+                ok = ptx::mbar_wait_warp(&bars[kPFull + (jg & 1)], (jg >> 1) & 1, abort_flag, S.status);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 if (lane == 0) {
                     const uint32_t v_base = ptx::smem_u32(smem + st * kStageBytes + kKHalfBytes);
-                    const uint32_t p_base = ptx::smem_u32(smem + kSmemP + (j & 1) * kPBytes);
+                    const uint32_t p_base = ptx::smem_u32(smem + kSmemP + (jg & 1) * kPBytes);
                     for (int ks = 0; ks < kChunk / 16; ++ks) {
                         const uint64_t ad = ptx::smem_desc(p_base + ks * 32, 16, 1024, ptx::kSwizzle128B);
                         const uint64_t bd = ptx::smem_desc(v_base + ks * 16 * 128, kSlabV, 1024, ptx::kSwizzle128B);
@@ -345,66 +449,60 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (ok && lane == 0) ptx::mma_commit2_mc(&bars[kOFinal], pair_mask);
             __syncwarp();
-            // consume the last stages' empty phases (the producer never waits on them) so that no
-            // commit is still pending when the CTA moves on
-            for (int jj = max(0, nchunks - kStages); ok && jj < nchunks; ++jj)
-                if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status))
-                    break;
-            if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
-            __syncwarp();
-        } else if (warp < 8) {
-            // ---------------- softmax: thread = (row, half) ----------------
-            const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-            {
-                // this half of the Q row -> tensor memory columns [384 + 64 wg, +64) as packed BF16
-                // (rows past the block's last token repeat its query; their results are not stored)
-                const uint4* qrow =
-                    reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + min(tok, n - 1)) * HQ + head) * kHeadDim) +
-                    16 * wg;
-                uint32_t r0[32], r1[32];
+        }
+        for (int jj = max(0, jg - kStages); ok && jj < jg; ++jj)
+            if (!ptx::mbar_wait_warp(&bars[kEmpty + jj % kStages], (jj / kStages) & 1, abort_flag, S.status)) break;
+        if (lane == 0) ptx::mma_commit2_mc(&bars[kDrain], pair_mask);   // after this warp's last MMA
+        __syncwarp();
+    } else if (warp < 8) {
+        // ---------------- softmax: thread = (row, half); then the item's rows to the workspace ----------------
+        const int row = 32 * (warp & 3) + lane;   // row of this CTA (lane of tensor memory)
+        const int wg = (warp >> 2) & 1;           // which half of keys / columns
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const bool issuer = (warp & 3) == 0 && lane == 0;   // this group's TMA stores
+        const float qs = a.qscale;
+        // this thread's half of the Q row of item y -> tensor memory columns [384 + 64 wg, +64) as
+        // packed BF16 (the caller makes sure every Q K^T that read the columns has completed)
+        auto load_q = [&](const Item& y) {
+            const int ty = kTileTok * (2 * y.p + pr) + (row >> 2);
+            const uint4* qrow = reinterpret_cast<const uint4*>(
+                                    a.q + ((size_t)(y.b * n + min(ty, n - 1)) * HQ + y.g * kQPerGroup + (row & 3)) *
+                                              kHeadDim) +
+                                16 * wg;
+            uint32_t r0[32], r1[32];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint4 v0 = __ldg(qrow + e), v1 = __ldg(qrow + 8 + e);
-                    r0[4 * e] = v0.x; r0[4 * e + 1] = v0.y; r0[4 * e + 2] = v0.z; r0[4 * e + 3] = v0.w;
-                    r1[4 * e] = v1.x; r1[4 * e + 1] = v1.y; r1[4 * e + 2] = v1.z; r1[4 * e + 3] = v1.w;
-                }
-                ptx::tmem_st32(lane_addr + kColQ + 64 * wg, r0);
-                ptx::tmem_st32(lane_addr + kColQ + 64 * wg + 32, r1);
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_at(&bars[kQReady], leader, rank);
-                // this half's part of q . w_g for the gate (the Q row is read again, from L1),
-                // while the first Q K^T runs
-                const float4* wrow = reinterpret_cast<const float4*>(smem + kSmemW) + ((row & 3) * kHeadDim + 128 * wg) / 4;
-                float gd = 0.f;
-#pragma unroll 2
-                for (int e = 0; e < 16; ++e) {
-                    const uint4 u = __ldg(qrow + e);
-                    const float4 w0 = wrow[2 * e], w1 = wrow[2 * e + 1];
-                    gd += __uint_as_float(u.x << 16) * w0.x + __uint_as_float(u.x & 0xffff0000u) * w0.y +
-                          __uint_as_float(u.y << 16) * w0.z + __uint_as_float(u.y & 0xffff0000u) * w0.w +
-                          __uint_as_float(u.z << 16) * w1.x + __uint_as_float(u.z & 0xffff0000u) * w1.y +
-                          __uint_as_float(u.w << 16) * w1.z + __uint_as_float(u.w & 0xffff0000u) * w1.w;
-                }
-                xch[kXchGate + wg * 128 + row] = gd;
-                ptx::named_bar_sync(1, kSoftmaxThreads);
-                if (wg == 0) {
-                    const float gsum = xch[kXchGate + row] + xch[kXchGate + 128 + row];
-                    xch[kXchGate + row] = tanhf(gsum + a.b_g[head]);
-                }
+            for (int e = 0; e < 8; ++e) {
+                const uint4 v0 = __ldg(qrow + e), v1 = __ldg(qrow + 8 + e);
+                r0[4 * e] = v0.x; r0[4 * e + 1] = v0.y; r0[4 * e + 2] = v0.z; r0[4 * e + 3] = v0.w;
+                r1[4 * e] = v1.x; r1[4 * e + 1] = v1.y; r1[4 * e + 2] = v1.z; r1[4 * e + 3] = v1.w;
             }
-            const int pq = s + tok;                    // query position
-            const int w = (s - 1) % S.R;               // slot of position s - 1 (s >= 1)
-            const int base_pos = s - 1 - w;
-            const float qs = a.qscale;
-            // which of keys [32 h, 32 h + 32) of chunk j this row sees, one bit per key
+            ptx::tmem_st32(lane_addr + kColQ + 64 * wg, r0);
+            ptx::tmem_st32(lane_addr + kColQ + 64 * wg + 32, r1);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_at(&bars[kQReady], leader, rank);
+        };
+        int jg = 0, kw = 0;
+        bool ok = true;
+        if (cluster < n_items) {
+            const Item y = make_item(S, cluster, npairs);
+            if (y.nchunks > 0) load_q(y);
+        }
+        for (int it = cluster; it < n_items; it += n_clusters) {
+            const Item x = make_item(S, it, npairs);
+            const int T = 2 * x.p + pr;
+            const int tok = kTileTok * T + (row >> 2);
+            const int pq = x.s + tok;                  // query position
+            const int w = (x.s - 1) % S.R;             // slot of position s - 1 (s >= 1)
+            const int base_pos = x.s - 1 - w;
+            // which of keys [32 h, 32 h + 32) of the item's chunk j this row sees, one bit per key
             auto vis32 = [&](int j, int h) -> uint32_t {
-                if (j < n_ring) {
+                if (j < x.n_ring) {
                     const int slot0 = kChunk * j + 32 * h;
-                    if (slot0 >= fill) return 0u;
-                    const bool all_valid = slot0 + 31 < fill;
-                    const bool wraps = (slot0 <= w) && (w < slot0 + 31) && (fill == S.R);
+                    if (slot0 >= x.fill) return 0u;
+                    const bool all_valid = slot0 + 31 < x.fill;
+                    const bool wraps = (slot0 <= w) && (w < slot0 + 31) && (x.fill == S.R);
                     const int first = wraps ? w + 1 : slot0;   // the oldest slot of the range
                     const int pk_min = base_pos + first - (first > w ? S.R : 0);
                     if (all_valid && pk_min >= pq - S.R) return 0xffffffffu;
@@ -413,30 +511,28 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) {
                         const int slot = slot0 + i;
                         const int pk = base_pos + slot - (slot > w ? S.R : 0);
-                        v |= (uint32_t)((slot < fill) && (pk >= pq - S.R)) << i;
+                        v |= (uint32_t)((slot < x.fill) && (pk >= pq - S.R)) << i;
                     }
                     return v;
                 }
-                if (j < n_ring + n_blk) {
-                    const int t0 = kChunk * (j - n_ring) + 32 * h;
+                if (j < x.n_ring + x.n_blk) {
+                    const int t0 = kChunk * (j - x.n_ring) + 32 * h;
                     if (t0 > tok || t0 >= n) return 0u;
                     const int last = min(tok, n - 1) - t0;     // keys t0 .. t0 + last are visible
                     return last >= 31 ? 0xffffffffu : ((2u << last) - 1u);
                 }
-                const int a0 = kChunk * (j - n_ring - n_blk) + 32 * h;
-                if (a0 >= bank_fill) return 0u;
-                return (bank_fill - a0 >= 32) ? 0xffffffffu : ((1u << (bank_fill - a0)) - 1u);
+                const int a0 = kChunk * (j - x.n_ring - x.n_blk) + 32 * h;
+                if (a0 >= x.bank_fill) return 0u;
+                return (x.bank_fill - a0 >= 32) ? 0xffffffffu : ((1u << (x.bank_fill - a0)) - 1u);
             };
-            // The two warpgroups take alternate chunks (this one: j = wg, wg + 2, ...), each a whole
-            // row of 64 keys. The reference max is handed from chunk to chunk through shared memory
-            // (named barrier 2 + wg: this group's value is ready); each group keeps its own row sum
-            // against the reference of its latest chunk.
+            // chunk loop: this group takes the item's chunks whose global index has parity wg
             const uint32_t scol = wg ? kColS1 : kColS0;
-            float m_w = -CUDART_INF_F;
-            bool ok = true;
-            for (int j = wg; j < nchunks; j += 2) {
+            float m_w = -CUDART_INF_F, l = 0.f;
+            const int jbase = jg;
+            for (int j = (wg - jbase) & 1; j < x.nchunks; j += 2) {
+                const int jj = jbase + j;               // global chunk index
                 const uint32_t vlo = vis32(j, 0), vhi = vis32(j, 1);
-                if (ok) ok = ptx::mbar_wait_warp(&bars[kSFull + wg], (j >> 1) & 1, abort_flag, S.status);
+                if (ok) ok = ptx::mbar_wait_warp(&bars[kSFull + wg], (jj >> 1) & 1, abort_flag, S.status);
                 ok = __all_sync(0xffffffffu, ok);
                 uint32_t sa[32], sb[32];   // keys [0, 32) and [32, 64)
                 if (ok) {
@@ -453,7 +549,6 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 }
 #define SR(i) __uint_as_float((i) < 32 ? sa[(i) & 31] : sb[(i) & 31])
                 const bool full = (vlo & vhi) == 0xffffffffu;
-                // the chunk's row max (raw scores; the scale is positive)
                 float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
                 if (full) {
 #pragma unroll
@@ -477,7 +572,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                     resc = (m_prev != -CUDART_INF_F);
                     m_new = mloc;
                 }
-                if (j + 1 < nchunks) {
+                if (j + 1 < x.nchunks) {
                     xch[row] = m_new;
                     ptx::named_bar_arrive(2 + wg, kSoftmaxThreads);
                 }
@@ -506,18 +601,17 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                         (i < 16 ? pa[i & 15] : pb[i & 15]) = pack_bf16(e0, e1);
                     }
                 }
+#undef SR
                 l = l * fac_l + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                // O may be rescaled only once P V of chunk j - 1 (the other group's) has completed,
-                // and this group's P buffer is free once P V of chunk j - 2 has; both are the
-                // stage barriers of those chunks.  P V runs in chunk order and this group saw
-                // P V of chunk j - 4 complete, so each barrier is at most one phase behind.
+                // O may be rescaled once P V of the previous chunk has completed; this group's P buffer
+                // is free once P V of global chunk jj - 2 has (possibly in the previous item: done then)
                 const bool rescale_warp = __any_sync(0xffffffffu, resc);
                 if (ok && rescale_warp)
-                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (j - 1) % kStages], ((j - 1) / kStages) & 1, abort_flag,
-                                             S.status);
-                if (ok && j >= 2)
-                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (j - 2) % kStages], ((j - 2) / kStages) & 1, abort_flag,
-                                             S.status);
+                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (jj - 1) % kStages], ((jj - 1) / kStages) & 1,
+                                             abort_flag, S.status);
+                if (ok && jj >= 2)
+                    ok = ptx::mbar_wait_warp(&bars[kEmpty + (jj - 2) % kStages], ((jj - 2) / kStages) & 1,
+                                             abort_flag, S.status);
                 if (!ok) continue;
                 if (rescale_warp) {
                     ptx::tc_fence_after();
@@ -534,7 +628,6 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     ptx::tmem_wait_st();
                 }
-#undef SR
                 // P row: 64 keys as BF16 = 128 bytes, 16-byte pieces swizzled by the row within its 8-row atom
                 uint8_t* prow = smem + kSmemP + wg * kPBytes + row * 128;
 #pragma unroll
@@ -549,7 +642,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive_at(&bars[kPFull + wg], leader, rank);
             }
-            // the row sum over both groups, on the last chunk's reference (references only grow)
+            jg = jbase + x.nchunks;
+            // the row sum over both groups, on the later reference (references only grow)
             xch[kXchEndL + wg * 128 + row] = l;
             xch[kXchEndM + wg * 128 + row] = m_w;
             ptx::named_bar_sync(1, kSoftmaxThreads);
@@ -562,115 +656,183 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 if (mo != -CUDART_INF_F) lt += lo * fast_ex2(mo - mf);
                 l = lt;
             }
-            const bool done = ok && ptx::mbar_wait_warp(&bars[kOFinal], 0, abort_flag, S.status);
-            // every MMA of the pair has completed (or the CTA gave up): the K/V stages are free
-            ptx::named_bar_sync(1, kSoftmaxThreads);
-            if (done) ptx::tc_fence_after();
-            const float inv = (done && l > 0.f) ? 1.f / l : 0.f;
-            uint8_t* rrow = smem + (size_t)row * 1024;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                if (done) {
+            ptx::named_bar_sync(1, kSoftmaxThreads);   // both groups have read the exchange of this item
+            const bool have_o =
+                ok && x.nchunks > 0 && ptx::mbar_wait_warp(&bars[kOFinal], kw & 1, abort_flag, S.status);
+            if (have_o) ptx::tc_fence_after();
+            // The next item's Q, so that its first Q K^T run during this drain: every Q K^T of this
+            // item has completed (O final), or it had none.
+            if (it + n_clusters < n_items) {
+                const Item y = make_item(S, it + n_clusters, npairs);
+                if (y.nchunks > 0) load_q(y);
+            }
+            const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
+            // This group's half of the rows, normalised (zeros for an empty bank), to the workspace in
+            // four steps of 32 columns: each thread writes its row into the group's P buffer (free:
+            // every P V of the item has completed) in the 128-byte swizzled layout, then one thread
+            // stores the [32 tokens][4 heads][32 dims] box with TMA (rows past the block are clipped);
+            // the next 32 columns are read from tensor memory while the box leaves the buffer.
+            uint8_t* stg = smem + kSmemP + wg * kPBytes;
+            uint8_t* srow = stg + row * 128;
+            const int bar_g = 4 + wg;
+            uint32_t o[32];
+            auto read_o = [&](int c) {
+                if (have_o) {
                     ptx::tmem_ld32(lane_addr + kColO + 128 * wg + 32 * c, o);
                     ptx::tmem_wait_ld();
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = 0u;
                 }
+            };
+            read_o(0);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int piece = 32 * wg + 8 * c + i;
-                    *reinterpret_cast<float4*>(rrow + ((piece ^ (row & 7)) << 4)) =
-                        make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                    __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<float4*>(srow + ((k ^ (row & 7)) << 4)) =
+                        make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                                    __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(bar_g, 128);
+                if (issuer) {
+                    tma_store_5d(&tm.ws, stg, 128 * wg + 32 * c, x.g * kQPerGroup, kTileTok * T, x.b, x.phase);
+                    ptx::bulk_commit();
                 }
+                if (c < 3) {
+                    read_o(c + 1);
+                    if (issuer) ptx::bulk_wait_read_all();   // the box has left the buffer
+                } else if (issuer) {
+                    // every box of the item is written: count this group's rows as done for the
+                    // commit of (sequence, group), which waits for all of them (high half of the
+                    // group's ticket word)
+                    bulk_wait_all();
+                    asm volatile("fence.proxy.async.global;\n" ::: "memory");
+                    __threadfence();
+                    atomicAdd(S.tickets + x.bg, 1u << 16);
+                }
+                ptx::named_bar_sync(bar_g, 128);
             }
-            ptx::fence_proxy_async_smem();   // the rows leave through a bulk copy
+            if (x.nchunks > 0) {
+                // O has been read by this warp: the pair's next item with chunks may overwrite it
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_at(&bars[kODrained], leader, rank);
+                ++kw;
+            }
         }
-    } else if (warp < 8) {
-        // nothing to read (empty bank): this CTA's rows are zero (and so is the anchor's gate term)
-        for (int c = 0; c < 32; ++c)
-            *reinterpret_cast<float4*>(smem + (size_t)row * 1024 + ((32 * wg + c) << 4)) = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (wg == 0) xch[kXchGate + row] = 0.f;
-        ptx::fence_proxy_async_smem();
     }
-
-    // ---------------- tail ----------------
-    // The local CTA of this tile combines rows [0, 64), the anchor CTA rows [64, 128): each first
-    // pushes the 64 rows the other one needs into that CTA's free stage area [128 KiB, 192 KiB).
-    // The cluster barrier below follows the producer warp's drain: this CTA's loads have landed and
-    // every tensor-core operation of its pair has completed, also after a wait ran out and the CTA
-    // abandoned its tile, so tensor memory may be freed and the stage area reused.
+    // every CTA of the cluster is done with its roles, and (the producer's drain) no load into it
+    // and no tensor-core operation of the pair is in flight; the softmax groups' workspace stores
+    // have completed
+    if (warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_all();
     __syncwarp();
     ptx::tc_fence_before();
-    ptx::cluster_sync();   // all four CTAs have their rows in shared memory; all tensor memory reads done
-    if (has_work && warp == kWarpQK) {
+    ptx::cluster_sync();
+    if (warp == kWarpQK) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc2(tmem, kTmemCols);
     }
-    const uint32_t peer = rank ^ 2u;
-    if (tid == 0) {
-        ptx::mbar_arrive_expect_tx(&bars[kXfer], 64 * 1024);
-        const uint32_t src = ptx::smem_u32(smem) + (uint32_t)(64 * (1 - phase)) * 1024u;
-        const uint32_t dst = ptx::cluster_map(ptx::smem_u32(smem) + 128u * 1024u, peer);
-        const uint32_t rbar = ptx::cluster_map(ptx::smem_u32(&bars[kXfer]), peer);
-        ptx::bulk_copy_to_peer(dst, src, 64 * 1024, rbar);
-        ptx::bulk_commit();
-    }
-    if (warp < 8) {
-        // one row per warp at a time: lane L makes output dims [8 L, 8 L + 8) (16 contiguous bytes)
-        // the partner's copy always comes: wait for it even after an abort, so that it has landed
-        // before this CTA exits
-        const bool got = ptx::mbar_wait_drain(&bars[kXfer], 0, S.status);
-#pragma unroll 2
-        for (int rr = 0; rr < 8; ++rr) {
-            const int lrow = 8 * warp + rr, crow = 64 * phase + lrow;
-            const int ctok = kTileTok * T + (crow >> 2), chead = g * kQPerGroup + (crow & 3);
-            const float gate = xch[kXchGate + crow];
-            const uint32_t off0 = (uint32_t)(((2 * lane) ^ (crow & 7)) << 4);
-            const uint32_t off1 = (uint32_t)(((2 * lane + 1) ^ (crow & 7)) << 4);
-            const uint8_t* mrow = smem + (size_t)crow * 1024;
-            const uint8_t* prow = smem + 128 * 1024 + (size_t)lrow * 1024;
-            const float4 m0 = *reinterpret_cast<const float4*>(mrow + off0);
-            const float4 m1 = *reinterpret_cast<const float4*>(mrow + off1);
-            float4 t0 = make_float4(0.f, 0.f, 0.f, 0.f), t1 = t0;
-            if (got) {
-                t0 = *reinterpret_cast<const float4*>(prow + off0);
-                t1 = *reinterpret_cast<const float4*>(prow + off1);
-            }
-            const float4 l0 = phase == 0 ? m0 : t0, l1 = phase == 0 ? m1 : t1;
-            const float4 c0 = phase == 0 ? t0 : m0, c1 = phase == 0 ? t1 : m1;
-            uint4 r;
-            r.x = pack_bf16(l0.x + gate * c0.x, l0.y + gate * c0.y);
-            r.y = pack_bf16(l0.z + gate * c0.z, l0.w + gate * c0.w);
-            r.z = pack_bf16(l1.x + gate * c1.x, l1.y + gate * c1.y);
-            r.w = pack_bf16(l1.z + gate * c1.z, l1.w + gate * c1.w);
-            if (ctok < n) reinterpret_cast<uint4*>(a.out + ((size_t)(b * n + ctok) * HQ + chead) * kHeadDim)[lane] = r;
-        }
-    }
-    if (tid == 0) ptx::bulk_wait_read_all();   // the outgoing copy has read this CTA's rows
+}
 
-    // Ring write.  The slot of block token i holds position s + i - R, which queries up to token i
-    // still read, so the rows of tile T (tokens [32 T, 32 T + 32)) may be written once tiles 0..T
-    // have finished reading the ring; both CTAs of a local pair are done here (the cluster barrier
-    // above follows every MMA of the pair).  Each local CTA marks its tile in bits 8.. of the
-    // group's ticket word and writes the rows of every tile its mark completes the prefix for (the
-    // count of finished CTAs is in bits 0..7).
-    if (phase == 0) {
-        int* range = tail_flag + 1;
-        if (tid == 0) {
-            __threadfence();
-            const unsigned bit = 1u << (8 + T);
-            const unsigned old = atomicOr(S.tickets + bg, bit) >> 8;
-            __threadfence();
-            range[0] = __ffs(~old) - 1;            // tiles done in a row before this mark
-            range[1] = __ffs(~(old | (bit >> 8))) - 1;   // and after it
+// ---- the commit: gate and combine, ring write, pending append, forced admit ----
+// (four CTAs per SM: the whole grid is resident at once at the bench's sizes)
+__global__ void __launch_bounds__(kCommitThreads, 4) prefill_commit_kernel(const __grid_constant__ PrefillArgs a) {
+    extern __shared__ __align__(16) uint8_t csmem[];
+    const LayerView& S = a.s;
+    // CTAs [0, B G) run the admits (first, so that they are scheduled first), then kCommitSlices
+    // slice CTAs per (sequence, group)
+    const int G = S.G, HQ = G * kQPerGroup, n = a.n_tok;
+    const int n_bg = S.B * G;
+    const int ci = blockIdx.x < n_bg ? (int)blockIdx.x : (int)blockIdx.x - n_bg;
+    const int bg = blockIdx.x < n_bg ? ci : ci / kCommitSlices;
+    const int slice = blockIdx.x < n_bg ? kCommitSlices : ci % kCommitSlices;
+    const int g = bg % G, b = bg / G;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int kP = kRowBytes / 16;           // 16-byte pieces per row
+    __shared__ int s_last;
+
+    // The counters as they were before this block; none is written before every CTA of the
+    // group has arrived (the last one writes them all).
+    const int32_t* cnt = S.counters + bg * 4;
+    const int s = max(cnt[0], 0);
+    const int bank_fill = min(max(cnt[1], 0), S.A);
+    const int pend_fill = min(max(cnt[2], 0), S.P);
+    const bool fits = pend_fill + n <= S.P;
+    const int np = fits ? pend_fill + n : pend_fill;
+    if (slice < kCommitSlices) {
+        const int per = (n + kCommitSlices - 1) / kCommitSlices;
+        const int t0 = min(n, slice * per), t1 = min(n, t0 + per);
+        // The slice's candidates to pending slots pend_fill + i: no kernel of this call reads them
+        // (the admit takes the block's candidates from the inputs), so this precedes the wait.
+        if (fits) {
+            copy_pieces<kCommitThreads, 4>((t1 - t0) * 2 * kP, [&](int e, const uint4*& from_p, uint4*& to_p) {
+                const int i = t0 + e / (2 * kP), c = e % (2 * kP);
+                const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
+                const size_t pd = ((size_t)bg * S.P + pend_fill + i) * kHeadDim;
+                if (c < kP) {
+                    from_p = reinterpret_cast<const uint4*>(a.cand_k + src) + c;
+                    to_p = reinterpret_cast<uint4*>(S.pend_k + pd) + c;
+                } else {
+                    from_p = reinterpret_cast<const uint4*>(a.cand_v + src) + (c - kP);
+                    to_p = reinterpret_cast<uint4*>(S.pend_v + pd) + (c - kP);
+                }
+            });
+            for (int i = t0 + tid; i < t1; i += kCommitThreads)
+                S.pend_score[(size_t)bg * S.P + pend_fill + i] = a.cand_score[(size_t)(b * n + i) * G + g];
+        }
+        // the gate of the slice's rows, tanh(q . w_g + b_g) with the unscaled query: one warp per row
+        float* gate = reinterpret_cast<float*>(csmem);
+        const int rows = (t1 - t0) * kQPerGroup;
+        for (int r = warp; r < rows; r += kCommitThreads / 32) {
+            const int t = t0 + r / kQPerGroup, head = g * kQPerGroup + r % kQPerGroup;
+            const uint4 qv = __ldg(reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + t) * HQ + head) * kHeadDim) + lane);
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim) + 2 * lane);
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim) + 2 * lane + 1);
+            float d = __uint_as_float(qv.x << 16) * w0.x + __uint_as_float(qv.x & 0xffff0000u) * w0.y +
+                      __uint_as_float(qv.y << 16) * w0.z + __uint_as_float(qv.y & 0xffff0000u) * w0.w +
+                      __uint_as_float(qv.z << 16) * w1.x + __uint_as_float(qv.z & 0xffff0000u) * w1.y +
+                      __uint_as_float(qv.w << 16) * w1.z + __uint_as_float(qv.w & 0xffff0000u) * w1.w;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            if (lane == 0) gate[r] = tanhf(d + a.b_g[head]);
         }
         __syncthreads();
-        const int t0 = min(n, kTileTok * range[0]), t1 = min(n, kTileTok * range[1]);
-        copy_pieces<kThreads, 8>((t1 - t0) * 2 * kRowBytes / 16, [&](int e, const uint4*& from_p, uint4*& to_p) {
-            constexpr int kP = kRowBytes / 16;
+        // every row of this (sequence, group) is in the workspace after this: 4 arrivals (2 CTAs x
+        // 2 softmax groups) per item, 2 npairs items
+        wait_rows(S, bg, 8 * ((n + 2 * kTileTok - 1) / (2 * kTileTok)));
+        const float* ws_local = a.ws;
+        const float* ws_anchor = a.ws + ws_rows_floats(S.B, n, HQ);
+        // out = local + gate * anchor for tokens [t0, t1) x the group's 4 heads, 4 dims per element;
+        // each thread issues the loads of kCommitUnroll elements before it combines and stores them
+        const int total = rows * (kHeadDim / 4);
+        for (int e0 = tid; e0 < total; e0 += kCommitUnroll * kCommitThreads) {
+            float4 lc[kCommitUnroll], an[kCommitUnroll];
+            size_t rowi[kCommitUnroll];
+            int d4[kCommitUnroll], rr[kCommitUnroll];
+#pragma unroll
+            for (int u = 0; u < kCommitUnroll; ++u) {
+                const int e = min(e0 + u * kCommitThreads, total - 1);
+                rr[u] = e / (kHeadDim / 4);
+                d4[u] = e % (kHeadDim / 4);
+                const int t = t0 + rr[u] / kQPerGroup, head = g * kQPerGroup + rr[u] % kQPerGroup;
+                rowi[u] = (size_t)(b * n + t) * HQ + head;
+                lc[u] = __ldcg(reinterpret_cast<const float4*>(ws_local + rowi[u] * kHeadDim) + d4[u]);
+                an[u] = __ldcg(reinterpret_cast<const float4*>(ws_anchor + rowi[u] * kHeadDim) + d4[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < kCommitUnroll; ++u) {
+                if (e0 + u * kCommitThreads < total) {
+                    const float gt = gate[rr[u]];
+                    uint2 o;
+                    o.x = pack_bf16(lc[u].x + gt * an[u].x, lc[u].y + gt * an[u].y);
+                    o.y = pack_bf16(lc[u].z + gt * an[u].z, lc[u].w + gt * an[u].w);
+                    reinterpret_cast<uint2*>(a.out + rowi[u] * kHeadDim)[d4[u]] = o;
+                }
+            }
+        }
+        // the block's K / V into ring slots (s + i) mod R (every read of the block is done)
+        copy_pieces<kCommitThreads, 4>((t1 - t0) * 2 * kP, [&](int e, const uint4*& from_p, uint4*& to_p) {
             const int i = t0 + e / (2 * kP), c = e % (2 * kP);
             const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
             const size_t dst = ((size_t)bg * S.R + (s + i) % S.R) * kHeadDim;
@@ -682,51 +844,85 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 to_p = reinterpret_cast<uint4*>(S.ring_v + dst) + (c - kP);
             }
         });
-    }
-
-    // This CTA's share of the candidates goes to pending now (nothing in this launch reads those
-    // slots before the last CTA's admit).
-    const bool fits = pend_fill + n <= S.P;
-    constexpr int kPieces = kRowBytes / 16;   // 32 per row
-    const int nct = gridDim.x, share = (n + nct - 1) / nct;
-    const int i0 = min(n, (int)blockIdx.x * share), i1 = min(n, i0 + share);
-    if (fits) {
-        copy_pieces<kThreads, 4>((i1 - i0) * 2 * kPieces, [&](int e, const uint4*& from_p, uint4*& to_p) {
-            const int i = i0 + e / (2 * kPieces), c = e % (2 * kPieces);
-            const size_t src = ((size_t)(b * n + i) * G + g) * kHeadDim;
-            const size_t pd = ((size_t)bg * S.P + pend_fill + i) * kHeadDim;
-            if (c < kPieces) {
-                from_p = reinterpret_cast<const uint4*>(a.cand_k + src) + c;
-                to_p = reinterpret_cast<uint4*>(S.pend_k + pd) + c;
-            } else {
-                from_p = reinterpret_cast<const uint4*>(a.cand_v + src) + (c - kPieces);
-                to_p = reinterpret_cast<uint4*>(S.pend_v + pd) + (c - kPieces);
+    } else {
+        // The forced admit over the committed bank and the pending buffer, the block's candidates
+        // included when they fit.  The competition reads scores only, and neither the attention
+        // launch nor the slices touch the bank's scores or the scores it reads, so this CTA does not
+        // wait: it writes the kept candidates' scores and leaves the list of (source, bank slot)
+        // pairs in the workspace for the copy launch, which moves the rows once the attention
+        // launch has read the bank.
+        const float* pscore = S.pend_score + (size_t)bg * S.P;
+        auto score_of = [&](int t) {
+            return t < pend_fill ? pscore[t] : a.cand_score[(size_t)(b * n + t - pend_fill) * G + g];
+        };
+        int n_adm = 0;
+        if (np > 0) n_adm = admit_select<kCommitThreads>(S, bg, bank_fill, np, csmem, score_of);
+        int* list = admit_list(a.ws, S.B, n, HQ, S.P, bg);
+        if (tid == 0) {
+            list[0] = n_adm;
+            list[1] = pend_fill;
+        }
+        if (n_adm > 0) {
+            const int* src = admit_src(csmem, S.A, S.P);
+            const int* dest = admit_dest(csmem, S.A, S.P);
+            for (int j = tid; j < n_adm; j += kCommitThreads) {
+                list[4 + j] = src[j];
+                list[4 + S.P + j] = dest[j];
+                S.bank_score[(size_t)bg * S.A + dest[j]] = score_of(src[j]);
             }
-        });
-        for (int i = i0 + tid; i < i1; i += kThreads)
-            S.pend_score[(size_t)bg * S.P + pend_fill + i] = a.cand_score[(size_t)(b * n + i) * G + g];
+        }
+        if (tid == 0 && !fits) atomicOr(S.status, (unsigned)RMA_STATUS_PREFILL_PENDING_OVERFLOW);
     }
+    // The last CTA of (b, g) to finish writes the counters (every CTA of the group read them
+    // before it arrived): pos advances by the block, the admit kept min(A, bank + candidates)
+    // records, and pending is empty.
     __threadfence();
     __syncthreads();
     if (tid == 0) {
         const unsigned old = atomicAdd(S.tickets + bg, 1u);
-        *tail_flag = (int)(old & 0xFFu) == 2 * ntiles - 1;
+        s_last = (old & 0xffffu) == (unsigned)kCommitSlices;
     }
     __syncthreads();
-    if (*tail_flag == 0) return;
-
-    // ---------------- last CTA of (b, g): the forced admit ----------------
-    __threadfence();
-    const int np = fits ? pend_fill + n : pend_fill;
-    __syncthreads();
-    if (tid == 0) {
+    if (s_last && tid == 0) {
+        __threadfence();
         int32_t* c = S.counters + bg * 4;
         c[0] = s + n;
-        c[2] = np;
-        if (!fits) atomicOr(S.status, (unsigned)RMA_STATUS_PREFILL_PENDING_OVERFLOW);
+        c[1] = min(S.A, bank_fill + np);
+        c[2] = 0;
+        S.tickets[bg] = 0u;
     }
-    if (np > 0) admit_group<kThreads, 16>(S, bg, bank_fill, np, smem);
-    if (tid == 0) S.tickets[bg] = 0u;
+}
+
+// ---- the admitted rows into the bank, once the attention launch has read it ----
+// kCopyParts CTAs per (sequence, group), each moving a share of the admit's list.
+constexpr int kCopyParts = 8;
+constexpr int kCopyThreads = 256;
+__global__ void __launch_bounds__(kCopyThreads) prefill_admit_copy_kernel(const __grid_constant__ PrefillArgs a) {
+    const LayerView& S = a.s;
+    const int G = S.G, HQ = G * kQPerGroup, n = a.n_tok;
+    const int bg = blockIdx.x / kCopyParts, part = blockIdx.x % kCopyParts;
+    const int g = bg % G, b = bg / G;
+    constexpr int kP = kRowBytes / 16;
+    // the commit launch (the lists) and, before it, the attention launch (every read of the bank)
+    // have completed
+    grid_dep_wait();
+    const int* list = admit_list(a.ws, S.B, n, HQ, S.P, bg);
+    const int n_adm = min(max(list[0], 0), S.P), pend_fill = list[1];
+    const int per = (n_adm + kCopyParts - 1) / kCopyParts;
+    const int j0 = min(n_adm, part * per), j1 = min(n_adm, j0 + per);
+    const int* src = list + 4;
+    const int* dest = list + 4 + S.P;
+    copy_pieces<kCopyThreads, 8>((j1 - j0) * 2 * kP, [&](int e, const uint4*& from_p, uint4*& to_p) {
+        const int j = j0 + e / (2 * kP), c = e % (2 * kP);
+        const bool kpart = c < kP;
+        const int piece = kpart ? c : c - kP;
+        const int t = src[j];
+        const uint16_t* from_row =
+            t < pend_fill ? (kpart ? S.pend_k : S.pend_v) + ((size_t)bg * S.P + t) * kHeadDim
+                          : (kpart ? a.cand_k : a.cand_v) + ((size_t)(b * n + t - pend_fill) * G + g) * kHeadDim;
+        from_p = reinterpret_cast<const uint4*>(from_row) + piece;
+        to_p = reinterpret_cast<uint4*>((kpart ? S.bank_k : S.bank_v) + ((size_t)bg * S.A + dest[j]) * kHeadDim) + piece;
+    });
 }
 
 // ---- host side: tensor maps through the driver entry point ----
@@ -764,22 +960,64 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d1, uint64_t d2, uint64
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The FP32 workspace [phase 2][b B][t n][head HQ][256] for TMA stores: boxes of 32 dims x 4 heads
+// x 32 tokens, 128-byte swizzle (the rows' 16-byte pieces permuted by row within 8-row groups).
+bool make_ws_map(CUtensorMap* m, void* ws, int HQ, int n, int B) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t row = (uint64_t)kHeadDim * 4;
+    const cuuint64_t dims[5] = {(cuuint64_t)kHeadDim, (cuuint64_t)HQ, (cuuint64_t)n, (cuuint64_t)B, 2};
+    const cuuint64_t strides[4] = {row, row * HQ, row * HQ * n, row * HQ * n * B};
+    const cuuint32_t box[5] = {32, (cuuint32_t)kQPerGroup, (cuuint32_t)kTileTok, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, ws, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of 2 attention CTAs that can be resident at once on the current device (cached per
+// device; half the SM count if the occupancy query fails).
+int resident_clusters() {
+    constexpr int kTracked = 64;
+    static std::atomic<int> cached[kTracked] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    if (dev >= 0 && dev < kTracked) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_attn_kernel, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        int sms = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        n = sms / 2 > 0 ? sms / 2 : 1;
+    }
+    if (dev >= 0 && dev < kTracked) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 }  // namespace
 
 size_t prefill_workspace_bytes(const rma_config& cfg, int n_tok) {
-    // the tile CTAs exchange their rows through distributed shared memory: no device scratch
-    (void)cfg;
-    (void)n_tok;
-    return 256;
+    // normalised local and anchor rows (FP32) of every (token, head) of the block
+    const int HQ = cfg.n_groups * cfg.q_per_group;
+    const size_t bytes = 2 * ws_rows_floats(cfg.batch, n_tok, HQ) * 4 +
+                         (size_t)cfg.batch * cfg.n_groups * admit_list_ints(cfg.pend_slots) * 4;
+    return (bytes + 255) / 256 * 256;
 }
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const LayerView& s = a.s;
     const int B = s.B, G = s.G, n = a.n_tok;
-    // tiles come in pairs (64 tokens, the last one possibly ragged); the ticket counts 2 * ntiles
-    // arrivals in 8 bits and marks one bit per tile in bits 8..15
     if (n < 1 || n > kMaxPrefillTokens || n > s.R) return cudaErrorNotSupported;
-    const int ntiles = kTilesPerCluster * ((n + kTilesPerCluster * kTileTok - 1) / (kTilesPerCluster * kTileTok));
+    const int npairs = (n + 2 * kTileTok - 1) / (2 * kTileTok);
+    const long long n_items = 2LL * B * G * npairs;
+    if (n_items > (1 << 30)) return cudaErrorNotSupported;
     Tmaps tm;
     const uint64_t row = (uint64_t)kHeadDim * 2;
     bool ok = make_map(&tm.k, a.k, G, (uint64_t)B * n, row, row * G, 1, kHalfKeys) &&
@@ -787,14 +1025,39 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
               make_map(&tm.ring_k, s.ring_k, s.R, (uint64_t)B * G, row, row * s.R, kHalfKeys, 1) &&
               make_map(&tm.ring_v, s.ring_v, s.R, (uint64_t)B * G, row, row * s.R, kChunk, 1) &&
               make_map(&tm.bank_k, s.bank_k, s.A, (uint64_t)B * G, row, row * s.A, kHalfKeys, 1) &&
-              make_map(&tm.bank_v, s.bank_v, s.A, (uint64_t)B * G, row, row * s.A, kChunk, 1);
+              make_map(&tm.bank_v, s.bank_v, s.A, (uint64_t)B * G, row, row * s.A, kChunk, 1) &&
+              make_ws_map(&tm.ws, a.ws, G * kQPerGroup, n, B);
     if (!ok) return cudaErrorInvalidValue;
-    static SmemLimit limit(reinterpret_cast<const void*>(prefill_kernel));
-    const cudaError_t e = limit.ensure(kSmemBytes);
+    static SmemLimit limit(reinterpret_cast<const void*>(prefill_attn_kernel));
+    cudaError_t e = limit.ensure(kSmemBytes);
     if (e != cudaSuccess) return e;
-    // grid x: clusters of 4 CTAs, one per pair of tiles; ranks (local, local, anchor, anchor)
-    prefill_kernel<<<dim3(2 * ntiles, G, B), kThreads, kSmemBytes, stream>>>(tm, a, ntiles);
-    return cudaGetLastError();
+    // one cluster of 2 per co-resident slot, each looping over its items
+    const int n_clusters = (int)std::min<long long>(n_items, resident_clusters());
+    prefill_attn_kernel<<<dim3(2 * n_clusters, 1, 1), kThreads, kSmemBytes, stream>>>(tm, a, npairs, (int)n_items);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // the commit, launched so that its CTAs may be scheduled while the attention launch finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((kCommitSlices + 1) * B * G), 1, 1);
+    cfg.blockDim = dim3(kCommitThreads, 1, 1);
+    cfg.dynamicSmemBytes = admit_scratch_bytes(s.A, s.P);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static SmemLimit climit(reinterpret_cast<const void*>(prefill_commit_kernel));
+    e = climit.ensure(cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaLaunchKernelEx(&cfg, prefill_commit_kernel, a);
+    if (e != cudaSuccess) return e;
+    // the copy of the admitted rows, launched the same way after the commit
+    cudaLaunchConfig_t ccfg = cfg;
+    ccfg.gridDim = dim3((unsigned)(kCopyParts * B * G), 1, 1);
+    ccfg.blockDim = dim3(kCopyThreads, 1, 1);
+    ccfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&ccfg, prefill_admit_copy_kernel, a);
 }
 
 }  // namespace rma

@@ -281,7 +281,13 @@ RMA_API int rma_admit(rma_state* st, int layer, int force, void* stream);
  *   w_g, b_g    as in rma_decode_step
  *   out         bf16 [batch][n_tok][n_groups*q_per_group][head_dim]  (written)
  *   ws          workspace of rma_workspace_bytes(st, n_tok) bytes
- * One launch: the admit runs inside it once every read of the block is done.
+ * Three launches on the stream: the attention (persistent, over work items of
+ * 64 tokens x one group x local window or bank), the commit (gate, combine,
+ * ring write, pending append, the admit's competition) and the copy of the
+ * admitted rows into the bank; the second and third may begin while the one
+ * before them finishes, and touch nothing it still reads.  The workspace holds
+ * the normalised local and anchor rows, 2 x batch x n_tok x n_groups x
+ * q_per_group x head_dim FP32, and the admit's lists.
  * n_tok is any length from 1 (RMA_ERR_INVALID_ARG below) to 256 and at most
  * ring_slots (RMA_ERR_UNSUPPORTED above): a prompt whose length is not a
  * multiple of pend_slots ends in a shorter block, and a block may follow

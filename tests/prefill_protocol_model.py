@@ -1,22 +1,27 @@
-"""A randomised model of the prefill kernel's barrier protocol (one CTA pair of one launch).
+"""A randomised model of the prefill attention kernel's barrier protocol (one cluster of 2 CTAs
+of one launch, looping over its work items).
 
-Test infrastructure: ``tests/test_prefill_protocol.py`` runs it on the CPU.  It mirrors the
-roles of ``rma_prefill.cu`` (the TMA producer of each CTA, the odd CTA's cleaner, the even CTA's
-two Q K^T issuers and its P V issuer, the two softmax groups of each CTA, and each CTA's tail)
-and the mbarriers they share.  Asynchronous work completes later, in a random order that keeps the
+Test infrastructure: ``tests/test_prefill_protocol.py`` runs it on the CPU.  It mirrors the roles
+of ``prefill_attn_kernel`` in ``rma_prefill.cu``: the TMA producer of each CTA, the odd CTA's
+cleaner, the even CTA's two Q K^T issuers and its P V issuer, the two softmax groups of each CTA
+(which also load each item's Q into tensor memory and drain its O), and each CTA's exit, with the
+mbarriers they share.  Asynchronous work completes later, in a random order that keeps the
 hardware's guarantees: TMA bytes land in any order; the pair's tensor pipe runs its MMAs in issue
 order; a tcgen05 commit arrives once every earlier MMA of its issuing thread is done.
 
-What it checks, over many random schedules:
-  * every parity wait is sound: it is made while its barrier has completed P or P + 1 phases (a
+What it checks, over many random schedules and item lists:
+  * every parity wait is sound: when it is issued its barrier has completed P or P + 1 phases (a
     barrier two phases ahead would let a parity wait pass on the wrong phase, and one whose phase
     P - 1 is still open would let it pass at once);
+  * tensor-memory and shared-memory hazards: Q of an item is written only when no Q K^T is queued
+    in the pipe; a Q K^T runs only on the Q of its own item; a P V of an item runs only after every
+    group of both CTAs has drained O of the previous item; a P V reads only a P its group wrote
+    for that chunk;
   * nothing deadlocks (an abort-aware wait that can never complete is timed out, as the kernel's
-    bounded wait would, and its CTA abandons its tile; a drain wait that can never complete is an
+    bounded wait would, and its CTA abandons its work; a drain wait that can never complete is an
     error);
-  * when a CTA passes the final cluster barrier (after which it frees tensor memory and reuses its
-    stage area), no TMA load into it, no MMA of its pair and no commit into its barriers is still
-    in flight.
+  * when a CTA passes the final cluster barrier (after which it frees tensor memory), no TMA load
+    into it, no MMA of its pair and no commit into its barriers is still in flight.
 
 ``abort_rate`` makes random abort-aware waits time out; ``async_bias`` sets how quickly the
 asynchronous work completes next to the warps; ``drain`` selects the kernel's drain (waits on the
@@ -52,10 +57,10 @@ class Hazard(Exception):
     pass
 
 
-def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, max_steps=400000):
-    """One launch of one CTA pair over n_chunks chunks (0 = an empty bank).  async_bias is the
-    chance that a scheduling step completes pending asynchronous work rather than advancing a role
-    (small values make copies and MMAs slow next to the warps)."""
+def run(items, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, max_steps=2_000_000):
+    """One cluster's launch over `items`, the chunk count of each of its work items in order (0 = an
+    item without chunks: an empty bank).  async_bias is the chance that a scheduling step completes
+    pending asynchronous work rather than advancing a role."""
     rng = random.Random(seed)
     E, O = 0, 1
     S = stages
@@ -64,17 +69,24 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
         bar[c] = {"Full": [Barrier(f"c{c}.Full{i}", 1) for i in range(S)],
                   "Empty": [Barrier(f"c{c}.Empty{i}", 1) for i in range(S)],
                   "SFull": [Barrier(f"c{c}.SFull{i}", 1) for i in range(2)],
-                  "OFinal": Barrier(f"c{c}.OFinal", 1), "Drain": Barrier(f"c{c}.Drain", 3),
-                  "Xfer": Barrier(f"c{c}.Xfer", 1)}
+                  "OFinal": Barrier(f"c{c}.OFinal", 1), "Drain": Barrier(f"c{c}.Drain", 3)}
     bar[E].update({"Peer": [Barrier(f"E.Peer{i}", 1) for i in range(S)], "QReady": Barrier("E.QReady", 16),
                    "PFull": [Barrier(f"E.PFull{i}", 8) for i in range(2)],
-                   "SFree": [Barrier(f"E.SFree{i}", 8) for i in range(2)]})
+                   "SFree": [Barrier(f"E.SFree{i}", 8) for i in range(2)],
+                   "ODrained": Barrier("E.ODrained", 16)})
     abort = {E: False, O: False}
     events = []                 # pending asynchronous completions: (kind, target cta, callable)
-    pipe = []                   # the pair's tensor pipe: ("mma", issuer) / ("commit", issuer, fn, targets)
+    pipe = []                   # the pair's tensor pipe: ("mma", issuer, check) / ("commit", issuer, fn, targets)
     issued = {E: 0, O: 0}       # chunks whose loads each producer issued
     passed_final = set()
     flags = set()
+    n_items = len(items)
+    base = [sum(items[:i]) for i in range(n_items + 1)]          # global index of each item's first chunk
+    with_chunks = [i for i in range(n_items) if items[i] > 0]
+    # tensor-memory contents: whose Q is in it (per CTA), which item's O each group has drained
+    q_of = {E: None, O: None}
+    drained = {(c, wg): -1 for c in (E, O) for wg in (0, 1)}   # last item with chunks whose O the group drained
+    p_of = {(c, wg): None for c in (E, O) for wg in (0, 1)}    # global chunk whose P is in the group's buffer
 
     def pipe_fire_commits():
         for op in list(pipe):
@@ -89,11 +101,13 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
         for i, op in enumerate(pipe):
             if op[0] == "mma":
                 pipe.pop(i)
+                if op[2] is not None:
+                    op[2]()
                 break
         pipe_fire_commits()
 
-    def mma(issuer):
-        pipe.append(("mma", issuer))
+    def mma(issuer, check=None):
+        pipe.append(("mma", issuer, check))
         events.append(("mma", None, pipe_step))
 
     def commit(issuer, key, idx=None):
@@ -103,135 +117,196 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
         pipe.append(("commit", issuer, fn, (E, O)))
         pipe_fire_commits()
 
-    # a wait is ("wait", cta, barrier, phase, drain?): drain waits ignore the abort flag
     def wait(c, b, phase, is_drain=False):
         return ("wait", c, b, phase, is_drain)
 
     # ---------------- roles ----------------
     def producer(c):
         ok = True
-        for j in range(n_chunks):
-            st = j % S
-            if j >= S:
-                ok = yield wait(c, bar[c]["Empty"][st], j // S - 1)
-                if not ok:
-                    break
-            bar[c]["Full"][st].arrive(1, tx=32)
-            events.append(("tma", c, lambda b=bar[c]["Full"][st]: b.complete_tx(32)))
-            issued[c] += 1
-        if drain and n_chunks > 0:
+        jg = 0
+        for it in range(n_items):
+            for j in range(items[it]):
+                st = jg % S
+                if jg >= S:
+                    ok = yield wait(c, bar[c]["Empty"][st], jg // S - 1)
+                    if not ok:
+                        break
+                bar[c]["Full"][st].arrive(1, tx=32)
+                events.append(("tma", c, lambda b=bar[c]["Full"][st]: b.complete_tx(32)))
+                issued[c] = jg + 1
+                jg += 1
+            if not ok:
+                break
+        if drain and issued[c] > 0:
             for jj in range(max(0, issued[c] - S), issued[c]):
                 yield wait(c, bar[c]["Full"][jj % S], jj // S, True)
+        if drain:
             yield wait(c, bar[c]["Drain"], 0, True)
         flags.add(("roles_done", c, "prod"))
 
     def cleaner():
-        for j in range(n_chunks):
-            st = j % S
-            ok = yield wait(O, bar[O]["Full"][st], j // S)
+        jg = 0
+        ok = True
+        for it in range(n_items):
+            for j in range(items[it]):
+                st = jg % S
+                ok = yield wait(O, bar[O]["Full"][st], jg // S)
+                if not ok:
+                    break
+                bar[E]["Peer"][st].arrive()
+                jg += 1
             if not ok:
                 break
-            bar[E]["Peer"][st].arrive()
-        for jj in range(max(0, n_chunks - S), n_chunks):
+        for jj in range(max(0, jg - S), jg):
+            if not ok:
+                break
             ok = yield wait(O, bar[O]["Empty"][jj % S], jj // S)
-            if not ok:
-                break
         flags.add(("roles_done", O, "clean"))
 
     def qk(mine):
-        ok = yield wait(E, bar[E]["QReady"], 0)
-        for j in range(mine, n_chunks, 2):
-            if not ok:
-                break
-            st = j % S
-            if j >= 2:
-                ok = yield wait(E, bar[E]["SFree"][j & 1], (j - 2) >> 1)
+        jg, kw = 0, 0
+        ok = True
+        for it in range(n_items):
+            if items[it] == 0:
+                continue
+            ok = yield wait(E, bar[E]["QReady"], kw)
+            kw += 1
+            for j in range(items[it]):
+                g = jg
+                jg += 1
                 if not ok:
                     break
-            ok = yield wait(E, bar[E]["Full"][st], j // S)
+                if (g & 1) != mine:
+                    continue
+                st = g % S
+                if g >= 2:
+                    ok = yield wait(E, bar[E]["SFree"][g & 1], (g - 2) >> 1)
+                    if not ok:
+                        break
+                ok = yield wait(E, bar[E]["Full"][st], g // S)
+                if not ok:
+                    break
+                ok = yield wait(E, bar[E]["Peer"][st], g // S)
+                if not ok:
+                    break
+
+                def check(it=it):
+                    if abort[E] or abort[O]:
+                        return
+                    for c in (E, O):
+                        if q_of[c] != it:
+                            raise Hazard(f"Q K^T of item {it} runs on CTA {c}'s Q of item {q_of[c]}")
+                mma(f"qk{mine}", check)
+                commit(f"qk{mine}", "SFull", g & 1)
             if not ok:
                 break
-            ok = yield wait(E, bar[E]["Peer"][st], j // S)
-            if not ok:
-                break
-            mma(f"qk{mine}")
-            commit(f"qk{mine}", "SFull", j & 1)
         if drain:
             commit(f"qk{mine}", "Drain")
         flags.add(("roles_done", E, f"qk{mine}"))
 
     def pv():
+        jg, kw = 0, 0
         ok = True
-        for j in range(n_chunks):
-            ok = yield wait(E, bar[E]["PFull"][j & 1], j >> 1)
-            if not ok:
-                break
-            mma("pv")
-            commit("pv", "Empty", j % S)
-        if ok:
-            commit("pv", "OFinal")
-            for jj in range(max(0, n_chunks - S), n_chunks):
-                ok = yield wait(E, bar[E]["Empty"][jj % S], jj // S)
+        for it in range(n_items):
+            if items[it] == 0:
+                continue
+            if kw >= 1:
+                ok = yield wait(E, bar[E]["ODrained"], kw - 1)
+            prev = with_chunks[kw - 1] if kw >= 1 else -1
+            kw += 1
+            for j in range(items[it]):
+                g = jg
+                jg += 1
                 if not ok:
                     break
+                ok = yield wait(E, bar[E]["PFull"][g & 1], g >> 1)
+                if not ok:
+                    break
+
+                def check(it=it, g=g, prev=prev):
+                    if abort[E] or abort[O]:
+                        return
+                    for c in (E, O):
+                        for wg in (0, 1):
+                            if drained[(c, wg)] < prev:
+                                raise Hazard(f"P V of item {it} runs before CTA {c} group {wg} drained O of item {prev}")
+                        if p_of[(c, g & 1)] != g:
+                            raise Hazard(f"P V of chunk {g} reads CTA {c}'s P of chunk {p_of[(c, g & 1)]}")
+                mma("pv", check)
+                commit("pv", "Empty", g % S)
+            if ok:
+                commit("pv", "OFinal")
+            else:
+                break
+        for jj in range(max(0, jg - S), jg):
+            if not ok:
+                break
+            ok = yield wait(E, bar[E]["Empty"][jj % S], jj // S)
         if drain:
             commit("pv", "Drain")
         flags.add(("roles_done", E, "pv"))
 
-    def group(c, wg):
+    def load_q(c, wg, it):
+        # the group's half of its rows' Q: no Q K^T may still be queued
+        if not (abort[E] or abort[O]) and any(op[0] == "mma" and op[1].startswith("qk") for op in pipe):
+            raise Hazard(f"CTA {c} group {wg} writes Q of item {it} while a Q K^T is queued")
+        flags.add(("q", c, wg, it))
+        if all(("q", cc, w, it) in flags for cc in (E, O) for w in (0, 1)):
+            q_of[E] = q_of[O] = it
         bar[E]["QReady"].arrive(4)
+
+    def group(c, wg):
         ok = True
-        for j in range(wg, n_chunks, 2):
-            if ok:
-                ok = yield wait(c, bar[c]["SFull"][wg], j >> 1)
-            if ok:
-                bar[E]["SFree"][wg].arrive(4)
-            if j >= 1:
-                yield ("flag", ("m", c, j - 1))          # the reference max handed over by the other group
-            flags.add(("m", c, j))
-            if not ok:
-                continue
-            if j >= 1 and rng.random() < 0.3:              # a rescale of O waits for P V of chunk j - 1
-                ok = yield wait(c, bar[c]["Empty"][(j - 1) % S], (j - 1) // S)
-            if ok and j >= 2:                              # this group's P buffer: P V of chunk j - 2 done
-                ok = yield wait(c, bar[c]["Empty"][(j - 2) % S], (j - 2) // S)
-            if not ok:
-                continue
-            bar[E]["PFull"][wg].arrive(4)
-
-    def softmax_end(c):
-        # both groups meet (named barrier 1), then the final O
-        yield ("flag", ("grpdone", c, 0))
-        yield ("flag", ("grpdone", c, 1))
-        ok = not abort[c]
-        if ok and n_chunks > 0:
-            ok = yield wait(c, bar[c]["OFinal"], 0)
-        flags.add(("roles_done", c, "softmax"))
-
-    def tail(c):
-        names = ["prod", "softmax"] + (["qk0", "qk1", "pv"] if c == E else ["clean"])
-        for other in (E, O):            # the cluster barrier: every role of both CTAs has arrived
-            for n in (["prod", "softmax"] + (["qk0", "qk1", "pv"] if other == E else ["clean"])):
-                yield ("flag", ("roles_done", other, n))
-        if not drain:
-            for _ in range(rng.randint(0, 3)):   # the fixed sleep: some completions land, maybe not all
+        jg, kw = 0, 0
+        if n_items and items[0] > 0:
+            load_q(c, wg, 0)
+        for it in range(n_items):
+            x = items[it]
+            for j in range(x):
+                g = jg + j
+                if (g & 1) != wg:
+                    continue
+                if ok:
+                    ok = yield wait(c, bar[c]["SFull"][wg], g >> 1)
+                if ok:
+                    bar[E]["SFree"][wg].arrive(4)
+                if j >= 1:
+                    yield ("flag", ("m", c, g - 1))          # the reference max handed over by the other group
+                flags.add(("m", c, g))
+                if not ok:
+                    continue
+                if j >= 1 and rng.random() < 0.3:              # a rescale of O waits for P V of chunk g - 1
+                    ok = yield wait(c, bar[c]["Empty"][(g - 1) % S], (g - 1) // S)
+                if ok and g >= 2:                              # this group's P buffer: P V of chunk g - 2 done
+                    ok = yield wait(c, bar[c]["Empty"][(g - 2) % S], (g - 2) // S)
+                if not ok:
+                    continue
+                p_of[(c, wg)] = g
+                bar[E]["PFull"][wg].arrive(4)
+            jg += x
+            # both groups meet (named barrier 1), then the final O of the item
+            flags.add(("met", c, wg, it))
+            yield ("flag", ("met", c, wg ^ 1, it))
+            have_o = False
+            if x > 0 and ok:
+                ok = yield wait(c, bar[c]["OFinal"], kw)
+                have_o = ok
+            # the next item's Q (every Q K^T of this item has completed), then the drain of O
+            if it + 1 < n_items and items[it + 1] > 0:
+                if ok:
+                    load_q(c, wg, it + 1)
+                else:
+                    bar[E]["QReady"].arrive(4)                # abandoned: the contents no longer matter
+            p_of[(c, wg)] = "drain"                          # the drain stages O in the group's P buffer
+            for _ in range(4):                               # four steps of 32 columns, each taking a while
                 yield ("sleep",)
-        passed_final.add(c)
-        # invariants: nothing still in flight into this CTA
-        if any(k == "tma" and t == c for (k, t, _) in events):
-            raise Hazard(f"CTA {c} passes the final barrier with a TMA load into it in flight")
-        if any(op[0] == "mma" for op in pipe):
-            raise Hazard(f"CTA {c} passes the final barrier with an MMA of its pair in flight")
-        if any(op[0] == "commit" for op in pipe):
-            raise Hazard(f"CTA {c} passes the final barrier with a commit into it pending")
-        # the exchange: the partner's copy into this CTA lands; wait for it before exiting
-        bar[c]["Xfer"].arrive(1, tx=64)
-        events.append(("xfer", c, lambda b=bar[c]["Xfer"]: b.complete_tx(64)))
-        yield wait(c, bar[c]["Xfer"], 0, True)
-        flags.add(("exit", c))
+            if x > 0:
+                if have_o:
+                    drained[(c, wg)] = it
+                bar[E]["ODrained"].arrive(4)
+                kw += 1
 
-    # group completion flags come from the group processes
-    def group_done(c, wg):
+    def softmax(c, wg):
         g = group(c, wg)
         res = None
         try:
@@ -239,18 +314,27 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
                 res = yield g.send(res) if res is not None else next(g)
         except StopIteration:
             pass
-        flags.add(("grpdone", c, wg))
+        flags.add(("roles_done", c, f"g{wg}"))
+
+    def tail(c):
+        for other in (E, O):            # the cluster barrier: every role of both CTAs has arrived
+            for n in (["prod", "g0", "g1"] + (["qk0", "qk1", "pv"] if other == E else ["clean"])):
+                yield ("flag", ("roles_done", other, n))
+        if not drain:
+            for _ in range(rng.randint(0, 3)):   # a fixed delay: some completions land, maybe not all
+                yield ("sleep",)
+        passed_final.add(c)
+        if any(k == "tma" and t == c for (k, t, _) in events):
+            raise Hazard(f"CTA {c} passes the final barrier with a TMA load into it in flight")
+        if any(op[0] == "mma" for op in pipe):
+            raise Hazard(f"CTA {c} passes the final barrier with an MMA of its pair in flight")
+        if any(op[0] == "commit" for op in pipe):
+            raise Hazard(f"CTA {c} passes the final barrier with a commit into it pending")
+        flags.add(("exit", c))
 
     procs = [("prod", E, producer(E)), ("prod", O, producer(O)), ("clean", O, cleaner()), ("qk0", E, qk(0)),
-             ("qk1", E, qk(1)), ("pv", E, pv()), ("g0", E, group_done(E, 0)), ("g1", E, group_done(E, 1)),
-             ("g0", O, group_done(O, 0)), ("g1", O, group_done(O, 1)), ("sm", E, softmax_end(E)),
-             ("sm", O, softmax_end(O)), ("tail", E, tail(E)), ("tail", O, tail(O))]
-    if n_chunks == 0:
-        # an empty bank: no tensor memory, no roles but the tails (the kernel skips everything)
-        procs = [p for p in procs if p[0] in ("tail",)]
-        for c in (E, O):
-            for n in ["prod", "softmax"] + (["qk0", "qk1", "pv"] if c == E else ["clean"]):
-                flags.add(("roles_done", c, n))
+             ("qk1", E, qk(1)), ("pv", E, pv()), ("g0", E, softmax(E, 0)), ("g1", E, softmax(E, 1)),
+             ("g0", O, softmax(O, 0)), ("g1", O, softmax(O, 1)), ("tail", E, tail(E)), ("tail", O, tail(O))]
     state = {p: None for p in procs}
     started = set()
 
@@ -273,7 +357,6 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
         runnable = [p for p in live if ready(state[p])]
         choices = [("p", p) for p in runnable] + [("e", i) for i in range(len(events))]
         if not choices:
-            # every process is blocked: the kernel's bounded waits run out; abort-aware ones give up
             blocked = [p for p in live if state[p] and state[p][0] == "wait" and not state[p][4]]
             if not blocked:
                 names = ", ".join(f"{p[0]}@{p[1]} {state[p][2].name if state[p][0] == 'wait' else state[p]}"
@@ -314,8 +397,6 @@ def run(n_chunks, seed, stages=5, abort_rate=0.0, drain=True, async_bias=0.5, ma
             continue
         nw = state[p]
         if nw is not None and nw[0] == "wait" and nw[2].done < nw[3] and not (abort[nw[1]] and not nw[4]):
-            # the phase before the awaited one is still open: its parity differs from the awaited
-            # phase's, so the hardware's parity wait would pass at once
             raise Hazard(f"{p[0]}@{p[1]} waits phase {nw[3]} of {nw[2].name}, which has completed only "
                          f"{nw[2].done}")
     return steps
