@@ -12,8 +12,9 @@
 //
 // Three launches.
 //
-// 1. prefill_attn_kernel, persistent: one cluster of 2 CTAs per pair of SMs,
-//    each cluster looping over work items.  An item is one (sequence, group,
+// 1. prefill_attn_kernel, persistent: clusters of 2 CTAs, one CTA per SM, as
+//    few as keep the most items per cluster at its minimum (the SMs left over
+//    run the commit of finished groups), each looping over work items.  An item is one (sequence, group,
 //    pair of tiles, phase): a tile is 32 tokens x the group's 4 query heads =
 //    128 query rows, the two tiles of a pair are the two CTAs of a tcgen05
 //    cta_group::2 MMA pair (M = 256; both read exactly the same keys, so each
@@ -169,6 +170,21 @@ __device__ __forceinline__ Item make_item(const LayerView& S, int it, int npairs
     return x;
 }
 
+// The items of cluster c out of n, nc clusters: at step k, item k nc + (c + 2 k) mod nc, a
+// permutation of each wave of nc items (so that a cluster's items do not all sit at the same
+// offset of their groups, which would give some clusters only the longest local items); a step
+// whose item lies past the last is skipped.
+struct ItemSeq {
+    int c, nc, n;
+    __device__ __forceinline__ int at(int k) const { return k * nc + (c + 2 * k) % nc; }
+    // the first step >= k that has an item, or -1
+    __device__ __forceinline__ int next(int k) const {
+        for (; (long long)k * nc < n; ++k)
+            if (at(k) < n) return k;
+        return -1;
+    }
+};
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&v);
@@ -250,6 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t rank = ptx::cluster_ctarank();
     const int pr = rank & 1;                     // 0: the pair's MMA-issuing CTA
     const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const ItemSeq seq{cluster, n_clusters, n_items};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = S.G, HQ = G * kQPerGroup, n = a.n_tok;
     const uint16_t pair_mask = 3u;
@@ -304,12 +321,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------- TMA producer: this CTA's half of every chunk of every item ----------------
         int jg = 0, issued = 0;
         bool ok = true;
-        for (int it = cluster; ok && it < n_items; it += n_clusters) {
-            const Item x = make_item(S, it, npairs);
-            if (it + n_clusters < n_items) {
+        for (int k = seq.next(0); ok && k >= 0; k = seq.next(k + 1)) {
+            const Item x = make_item(S, seq.at(k), npairs);
+            if (seq.next(k + 1) >= 0) {
                 // the next item's query rows of this CTA into L2 (one token's 4 heads per lane): its
                 // softmax threads load them when that item starts
-                const Item y = make_item(S, it + n_clusters, npairs);
+                const Item y = make_item(S, seq.at(seq.next(k + 1)), npairs);
                 const int t = kTileTok * (2 * y.p + pr) + lane;
                 if (t < n) prefetch_l2(a.q + ((size_t)(y.b * n + t) * HQ + y.g * kQPerGroup) * kHeadDim, kQPerGroup * kRowBytes);
             }
@@ -358,8 +375,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ---------------- odd CTA: check its half landed, clear stale rows, tell the even CTA ----------------
         int jg = 0;
         bool ok = true;
-        for (int it = cluster; ok && it < n_items; it += n_clusters) {
-            const Item x = make_item(S, it, npairs);
+        for (int k = seq.next(0); ok && k >= 0; k = seq.next(k + 1)) {
+            const Item x = make_item(S, seq.at(k), npairs);
             for (int j = 0; j < x.nchunks; ++j, ++jg) {
                 const int st = jg % kStages;
                 if (!ptx::mbar_wait_warp(&bars[kFull + st], (jg / kStages) & 1, abort_flag, S.status)) {
@@ -380,8 +397,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int mine = warp == kWarpQK ? 0 : 1;
         int jg = 0, kw = 0;
         bool ok = true;
-        for (int it = cluster; ok && it < n_items; it += n_clusters) {
-            const Item x = make_item(S, it, npairs);
+        for (int k = seq.next(0); ok && k >= 0; k = seq.next(k + 1)) {
+            const Item x = make_item(S, seq.at(k), npairs);
             if (x.nchunks == 0) continue;        // an empty bank: no Q K^T, and its Q is not loaded
             // Q of this item is in tensor memory (phase kw of kQReady).  Both issuers wait for every
             // phase, in order, even in an item where one of them has no chunk: a parity wait on a
@@ -424,8 +441,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // kQReady, kOFinal and kODrained count only the items that have chunks (kw of them so far)
         int jg = 0, kw = 0;
         bool ok = true;
-        for (int it = cluster; ok && it < n_items; it += n_clusters) {
-            const Item x = make_item(S, it, npairs);
+        for (int k = seq.next(0); ok && k >= 0; k = seq.next(k + 1)) {
+            const Item x = make_item(S, seq.at(k), npairs);
             if (x.nchunks == 0) continue;
             // the previous item's O has been read by both CTAs before this item's first P V
             if (kw >= 1) ok = ptx::mbar_wait_warp(&bars[kODrained], (kw - 1) & 1, abort_flag, S.status);
@@ -485,12 +502,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         };
         int jg = 0, kw = 0;
         bool ok = true;
-        if (cluster < n_items) {
-            const Item y = make_item(S, cluster, npairs);
+        if (seq.next(0) >= 0) {
+            const Item y = make_item(S, seq.at(seq.next(0)), npairs);
             if (y.nchunks > 0) load_q(y);
         }
-        for (int it = cluster; it < n_items; it += n_clusters) {
-            const Item x = make_item(S, it, npairs);
+        for (int k = seq.next(0); k >= 0; k = seq.next(k + 1)) {
+            const Item x = make_item(S, seq.at(k), npairs);
             const int T = 2 * x.p + pr;
             const int tok = kTileTok * T + (row >> 2);
             const int pq = x.s + tok;                  // query position
@@ -662,8 +679,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (have_o) ptx::tc_fence_after();
             // The next item's Q, so that its first Q K^T run during this drain: every Q K^T of this
             // item has completed (O final), or it had none.
-            if (it + n_clusters < n_items) {
-                const Item y = make_item(S, it + n_clusters, npairs);
+            if (seq.next(k + 1) >= 0) {
+                const Item y = make_item(S, seq.at(seq.next(k + 1)), npairs);
                 if (y.nchunks > 0) load_q(y);
             }
             const float inv = (have_o && l > 0.f) ? 1.f / l : 0.f;
@@ -1032,7 +1049,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     cudaError_t e = limit.ensure(kSmemBytes);
     if (e != cudaSuccess) return e;
     // one cluster of 2 per co-resident slot, each looping over its items
-    const int n_clusters = (int)std::min<long long>(n_items, resident_clusters());
+    // As many clusters as keep the most items per cluster at its minimum: the SMs left over run the
+    // commit of the groups that are done while the last items run.
+    const long long per_cluster = (n_items + resident_clusters() - 1) / resident_clusters();
+    const int n_clusters = (int)((n_items + per_cluster - 1) / per_cluster);
     prefill_attn_kernel<<<dim3(2 * n_clusters, 1, 1), kThreads, kSmemBytes, stream>>>(tm, a, npairs, (int)n_items);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
