@@ -67,6 +67,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -102,7 +103,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
 constexpr int kCommitThreads = 256;
 constexpr int kCommitSlices = 16;                     // slice CTAs per (sequence, group) in the commit
-constexpr int kCommitUnroll = 4;                      // combine elements a thread loads before it stores
+constexpr int kCommitUnroll = 4;                      // combine tokens a thread loads before it stores
+constexpr int kCommitMaxTok = 16;                     // tokens of one slice: 256 / kCommitSlices
+static_assert(kMaxPrefillTokens <= kCommitSlices * kCommitMaxTok, "a slice holds at most kCommitMaxTok tokens");
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
@@ -753,7 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ---- the commit: gate and combine, ring write, pending append, forced admit ----
-// (four CTAs per SM: the whole grid is resident at once at the bench's sizes)
+// (three CTAs per SM)
 __global__ void __launch_bounds__(kCommitThreads, 4) prefill_commit_kernel(const __grid_constant__ PrefillArgs a) {
     extern __shared__ __align__(16) uint8_t csmem[];
     const LayerView& S = a.s;
@@ -798,53 +801,72 @@ __global__ void __launch_bounds__(kCommitThreads, 4) prefill_commit_kernel(const
             for (int i = t0 + tid; i < t1; i += kCommitThreads)
                 S.pend_score[(size_t)bg * S.P + pend_fill + i] = a.cand_score[(size_t)(b * n + i) * G + g];
         }
-        // the gate of the slice's rows, tanh(q . w_g + b_g) with the unscaled query: one warp per row
-        float* gate = reinterpret_cast<float*>(csmem);
+        // The gate of the slice's rows, tanh(q . w_g + b_g) with the unscaled query: the group's 4
+        // w_g rows staged in shared memory, then each warp takes rows warp, warp + 8, ... with
+        // every query load issued before the first dot product (a lane holds 8 dims of a row).
+        float* gate = reinterpret_cast<float*>(csmem);                     // [rows]
+        float* wsh = reinterpret_cast<float*>(csmem) + 4 * kCommitMaxTok;    // [4][256]
         const int rows = (t1 - t0) * kQPerGroup;
-        for (int r = warp; r < rows; r += kCommitThreads / 32) {
-            const int t = t0 + r / kQPerGroup, head = g * kQPerGroup + r % kQPerGroup;
-            const uint4 qv = __ldg(reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + t) * HQ + head) * kHeadDim) + lane);
-            const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim) + 2 * lane);
-            const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)head * kHeadDim) + 2 * lane + 1);
-            float d = __uint_as_float(qv.x << 16) * w0.x + __uint_as_float(qv.x & 0xffff0000u) * w0.y +
-                      __uint_as_float(qv.y << 16) * w0.z + __uint_as_float(qv.y & 0xffff0000u) * w0.w +
-                      __uint_as_float(qv.z << 16) * w1.x + __uint_as_float(qv.z & 0xffff0000u) * w1.y +
-                      __uint_as_float(qv.w << 16) * w1.z + __uint_as_float(qv.w & 0xffff0000u) * w1.w;
+        reinterpret_cast<float4*>(wsh)[tid] =
+            __ldg(reinterpret_cast<const float4*>(a.w_g + (size_t)g * kQPerGroup * kHeadDim) + tid);
+        __syncthreads();
+        {
+            constexpr int kRowsPerWarp = 4 * kCommitMaxTok / (kCommitThreads / 32);
+            uint4 qv[kRowsPerWarp];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-            if (lane == 0) gate[r] = tanhf(d + a.b_g[head]);
+            for (int u = 0; u < kRowsPerWarp; ++u) {
+                const int r = warp + 8 * u;
+                const int t = t0 + min(r, rows - 1) / kQPerGroup, head = g * kQPerGroup + min(r, rows - 1) % kQPerGroup;
+                qv[u] = rows > 0 ? __ldg(reinterpret_cast<const uint4*>(a.q + ((size_t)(b * n + t) * HQ + head) * kHeadDim) + lane)
+                                 : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kRowsPerWarp; ++u) {
+                const int r = warp + 8 * u;
+                const int h = r % kQPerGroup;
+                const float4 w0 = reinterpret_cast<const float4*>(wsh + h * kHeadDim)[2 * lane];
+                const float4 w1 = reinterpret_cast<const float4*>(wsh + h * kHeadDim)[2 * lane + 1];
+                const uint4 q4 = qv[u];
+                float d = __uint_as_float(q4.x << 16) * w0.x + __uint_as_float(q4.x & 0xffff0000u) * w0.y +
+                          __uint_as_float(q4.y << 16) * w0.z + __uint_as_float(q4.y & 0xffff0000u) * w0.w +
+                          __uint_as_float(q4.z << 16) * w1.x + __uint_as_float(q4.z & 0xffff0000u) * w1.y +
+                          __uint_as_float(q4.w << 16) * w1.z + __uint_as_float(q4.w & 0xffff0000u) * w1.w;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+                if (lane == 0 && r < rows) gate[r] = tanhf(d + a.b_g[g * kQPerGroup + h]);
+            }
         }
         __syncthreads();
         // every row of this (sequence, group) is in the workspace after this: 4 arrivals (2 CTAs x
         // 2 softmax groups) per item, 2 npairs items
         wait_rows(S, bg, 8 * ((n + 2 * kTileTok - 1) / (2 * kTileTok)));
-        const float* ws_local = a.ws;
-        const float* ws_anchor = a.ws + ws_rows_floats(S.B, n, HQ);
-        // out = local + gate * anchor for tokens [t0, t1) x the group's 4 heads, 4 dims per element;
-        // each thread issues the loads of kCommitUnroll elements before it combines and stores them
-        const int total = rows * (kHeadDim / 4);
-        for (int e0 = tid; e0 < total; e0 += kCommitUnroll * kCommitThreads) {
-            float4 lc[kCommitUnroll], an[kCommitUnroll];
-            size_t rowi[kCommitUnroll];
-            int d4[kCommitUnroll], rr[kCommitUnroll];
+        // out = local + gate * anchor: thread (head r0, dims 4 d4 .. 4 d4 + 3) over the slice's
+        // tokens, kCommitUnroll tokens' loads in flight before it combines and stores them
+        {
+            const int r0 = tid >> 6, d4 = tid & 63;
+            const size_t row0 = (size_t)(b * n + t0) * HQ + g * kQPerGroup + r0;
+            const size_t step = (size_t)HQ * (kHeadDim / 4);   // float4 (and 4-value output) pieces per token
+            const float4* lb = reinterpret_cast<const float4*>(a.ws + row0 * kHeadDim) + d4;
+            const float4* ab = reinterpret_cast<const float4*>(a.ws + ws_rows_floats(S.B, n, HQ) + row0 * kHeadDim) + d4;
+            uint2* ob = reinterpret_cast<uint2*>(a.out + row0 * kHeadDim) + d4;
+            const int ntok = t1 - t0;
+            for (int k0 = 0; k0 < ntok; k0 += kCommitUnroll) {
+                float4 lc[kCommitUnroll], an[kCommitUnroll];
 #pragma unroll
-            for (int u = 0; u < kCommitUnroll; ++u) {
-                const int e = min(e0 + u * kCommitThreads, total - 1);
-                rr[u] = e / (kHeadDim / 4);
-                d4[u] = e % (kHeadDim / 4);
-                const int t = t0 + rr[u] / kQPerGroup, head = g * kQPerGroup + rr[u] % kQPerGroup;
-                rowi[u] = (size_t)(b * n + t) * HQ + head;
-                lc[u] = __ldcg(reinterpret_cast<const float4*>(ws_local + rowi[u] * kHeadDim) + d4[u]);
-                an[u] = __ldcg(reinterpret_cast<const float4*>(ws_anchor + rowi[u] * kHeadDim) + d4[u]);
-            }
+                for (int u = 0; u < kCommitUnroll; ++u) {
+                    const int k = min(k0 + u, ntok - 1);
+                    lc[u] = __ldcg(lb + k * step);
+                    an[u] = __ldcg(ab + k * step);
+                }
 #pragma unroll
-            for (int u = 0; u < kCommitUnroll; ++u) {
-                if (e0 + u * kCommitThreads < total) {
-                    const float gt = gate[rr[u]];
-                    uint2 o;
-                    o.x = pack_bf16(lc[u].x + gt * an[u].x, lc[u].y + gt * an[u].y);
-                    o.y = pack_bf16(lc[u].z + gt * an[u].z, lc[u].w + gt * an[u].w);
-                    reinterpret_cast<uint2*>(a.out + rowi[u] * kHeadDim)[d4[u]] = o;
+                for (int u = 0; u < kCommitUnroll; ++u) {
+                    if (k0 + u < ntok) {
+                        const float gt = gate[(k0 + u) * kQPerGroup + r0];
+                        uint2 o;
+                        o.x = pack_bf16(lc[u].x + gt * an[u].x, lc[u].y + gt * an[u].y);
+                        o.y = pack_bf16(lc[u].z + gt * an[u].z, lc[u].w + gt * an[u].w);
+                        ob[(k0 + u) * step] = o;
+                    }
                 }
             }
         }
@@ -1060,7 +1082,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((kCommitSlices + 1) * B * G), 1, 1);
     cfg.blockDim = dim3(kCommitThreads, 1, 1);
-    cfg.dynamicSmemBytes = admit_scratch_bytes(s.A, s.P);
+    // the admit's scratch, or the slices' gate and w_g rows if a small state makes that larger
+    cfg.dynamicSmemBytes = std::max(admit_scratch_bytes(s.A, s.P), (size_t)(4 * kCommitMaxTok + 4 * kHeadDim) * 4);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
