@@ -102,9 +102,9 @@ constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 256, kColS1 = 320, kColQ = 384;
 constexpr int kCommitThreads = 256;
-constexpr int kCommitSlices = 16;                     // slice CTAs per (sequence, group) in the commit
+constexpr int kCommitSlices = 32;                     // slice CTAs per (sequence, group) in the commit
 constexpr int kCommitUnroll = 4;                      // combine tokens a thread loads before it stores
-constexpr int kCommitMaxTok = 16;                     // tokens of one slice: 256 / kCommitSlices
+constexpr int kCommitMaxTok = 8;                      // tokens of one slice: 256 / kCommitSlices
 static_assert(kMaxPrefillTokens <= kCommitSlices * kCommitMaxTok, "a slice holds at most kCommitMaxTok tokens");
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
