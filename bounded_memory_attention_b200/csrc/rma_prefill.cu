@@ -36,10 +36,10 @@
 //        through shared memory (moved only when a chunk's max exceeds it by more
 //        than 2^8, O rescaled then).  At the end of the item they write the
 //        normalised rows (FP32) to the workspace, 32 columns at a time through
-//        their P buffer and a TMA store, and go on to the next item, whose first
-//        K/V chunks are already loaded and whose query rows the TMA warp has
-//        asked L2 for; the P V issuer starts that item's P V once both CTAs have
-//        read O.
+//        their P buffer and a TMA store per warp (its 32 rows), and go on to the
+//        next item, whose first K/V chunks are already loaded and whose query
+//        rows the TMA warp has asked L2 for; the P V issuer starts that item's
+//        P V once both CTAs have read O.
 //    Every barrier phase follows a chunk counter (or a counter of the items
 //    that have chunks) running on across items.  A group's counters are
 //    constant while any of its items runs: the second launch writes them only
@@ -49,8 +49,9 @@
 //    group), slice CTAs append their tokens' candidates to pending and compute
 //    the gate tanh(q . w_g + b_g) of their rows at once (neither is read by the
 //    first launch), wait until every item of their group has stored its rows
-//    (the items count themselves in the high half of the group's ticket word
-//    once their TMA stores have completed; items run in group-major order, so
+//    (each softmax warp counts its rows of an item in the high half of the
+//    group's ticket word once its TMA stores have completed; items run in
+//    group-major order, so
 //    most groups are done well before the last), then combine out = local +
 //    gate * anchor in FP32, rounded once to BF16, and write the block's K/V into
 //    the ring (every read of the group's ring is done); one CTA runs the forced
@@ -479,7 +480,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int row = 32 * (warp & 3) + lane;   // row of this CTA (lane of tensor memory)
         const int wg = (warp >> 2) & 1;           // which half of keys / columns
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        const bool issuer = (warp & 3) == 0 && lane == 0;   // this group's TMA stores
         const float qs = a.qscale;
         // this thread's half of the Q row of item y -> tensor memory columns [384 + 64 wg, +64) as
         // packed BF16 (the caller makes sure every Q K^T that read the columns has completed)
@@ -692,9 +692,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // every P V of the item has completed) in the 128-byte swizzled layout, then one thread
             // stores the [32 tokens][4 heads][32 dims] box with TMA (rows past the block are clipped);
             // the next 32 columns are read from tensor memory while the box leaves the buffer.
-            uint8_t* stg = smem + kSmemP + wg * kPBytes;
-            uint8_t* srow = stg + row * 128;
-            const int bar_g = 4 + wg;
+            // each warp stores its own 32 rows (8 tokens x 4 heads) from its 4 KB of the group's P buffer
+            uint8_t* stg = smem + kSmemP + wg * kPBytes + (warp & 3) * 4096;
+            uint8_t* srow = stg + lane * 128;
             uint32_t o[32];
             auto read_o = [&](int c) {
                 if (have_o) {
@@ -708,31 +708,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             read_o(0);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                if (c > 0) {
+                    if (lane == 0) ptx::bulk_wait_read_all();   // the previous box has left the buffer
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<float4*>(srow + ((k ^ (row & 7)) << 4)) =
+                    *reinterpret_cast<float4*>(srow + ((k ^ (lane & 7)) << 4)) =
                         make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
                                     __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
                 ptx::fence_proxy_async_smem();
-                ptx::named_bar_sync(bar_g, 128);
-                if (issuer) {
-                    tma_store_5d(&tm.ws, stg, 128 * wg + 32 * c, x.g * kQPerGroup, kTileTok * T, x.b, x.phase);
+                __syncwarp();
+                if (lane == 0 && kTileTok * T + 8 * (warp & 3) < n) {   // rows past the block are not stored
+                    tma_store_5d(&tm.ws, stg, 128 * wg + 32 * c, x.g * kQPerGroup, kTileTok * T + 8 * (warp & 3),
+                                 x.b, x.phase);
                     ptx::bulk_commit();
                 }
-                if (c < 3) {
-                    read_o(c + 1);
-                    if (issuer) ptx::bulk_wait_read_all();   // the box has left the buffer
-                } else if (issuer) {
-                    // every box of the item is written: count this group's rows as done for the
-                    // commit of (sequence, group), which waits for all of them (high half of the
-                    // group's ticket word)
-                    bulk_wait_all();
-                    asm volatile("fence.proxy.async.global;\n" ::: "memory");
-                    __threadfence();
-                    atomicAdd(S.tickets + x.bg, 1u << 16);
-                }
-                ptx::named_bar_sync(bar_g, 128);
+                if (c < 3) read_o(c + 1);
             }
+            if (lane == 0) {
+                // every box of this warp is written (and its rows of the P buffer are free): count
+                // them as done for the commit of (sequence, group), which waits for all 16 warps of
+                // the pair per item (high half of the group's ticket word)
+                bulk_wait_all();
+                asm volatile("fence.proxy.async.global;\n" ::: "memory");
+                __threadfence();
+                atomicAdd(S.tickets + x.bg, 1u << 16);
+            }
+            __syncwarp();
             if (x.nchunks > 0) {
                 // O has been read by this warp: the pair's next item with chunks may overwrite it
                 ptx::tc_fence_before();
@@ -837,9 +840,9 @@ __global__ void __launch_bounds__(kCommitThreads, 4) prefill_commit_kernel(const
             }
         }
         __syncthreads();
-        // every row of this (sequence, group) is in the workspace after this: 4 arrivals (2 CTAs x
-        // 2 softmax groups) per item, 2 npairs items
-        wait_rows(S, bg, 8 * ((n + 2 * kTileTok - 1) / (2 * kTileTok)));
+        // every row of this (sequence, group) is in the workspace after this: 16 arrivals (2 CTAs x
+        // 8 softmax warps) per item, 2 npairs items
+        wait_rows(S, bg, 32 * ((n + 2 * kTileTok - 1) / (2 * kTileTok)));
         // out = local + gate * anchor: thread (head r0, dims 4 d4 .. 4 d4 + 3) over the slice's
         // tokens, kCommitUnroll tokens' loads in flight before it combines and stores them
         {
@@ -1007,7 +1010,7 @@ bool make_ws_map(CUtensorMap* m, void* ws, int HQ, int n, int B) {
     const uint64_t row = (uint64_t)kHeadDim * 4;
     const cuuint64_t dims[5] = {(cuuint64_t)kHeadDim, (cuuint64_t)HQ, (cuuint64_t)n, (cuuint64_t)B, 2};
     const cuuint64_t strides[4] = {row, row * HQ, row * HQ * n, row * HQ * n * B};
-    const cuuint32_t box[5] = {32, (cuuint32_t)kQPerGroup, (cuuint32_t)kTileTok, 1, 1};
+    const cuuint32_t box[5] = {32, (cuuint32_t)kQPerGroup, (cuuint32_t)(kTileTok / 4), 1, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, ws, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
