@@ -109,3 +109,31 @@ def test_a_producer_reusing_a_stage_one_phase_early_is_caught():
         except ns["Hazard"]:
             caught += 1
     assert caught > 0
+
+
+def test_commit_hand_off_through_the_ticket_word():
+    """The prefill call's cross-launch hand-off (``prefill_commit_model.py``): slices read a group's
+    rows only after every item stored them, the counters change only after every item finished, and
+    the word is zero after the call, over random interleavings and shapes."""
+    import prefill_commit_model as cm
+    for seed in range(200):
+        r = random.Random(seed)
+        cm.run(n_groups=r.choice([1, 3, 8]), npairs=r.choice([1, 2, 4]), n_clusters=r.choice([1, 5, 16, 64]),
+               slices=r.choice([1, 4, 32]), seed=seed)
+
+
+def test_a_slice_waiting_for_too_few_arrivals_is_caught():
+    """A planted mistake: the slices' wait counts one softmax group per item instead of every warp."""
+    import prefill_commit_model as cm
+    src = open(cm.__file__).read()
+    bad = src.replace("    need = warps_per_item * per_group", "    need = 2 * per_group")
+    assert bad != src
+    ns = {}
+    exec(compile(bad, "planted_commit_model", "exec"), ns)
+    caught = 0
+    for seed in range(50):
+        try:
+            ns["run"](n_groups=3, npairs=2, n_clusters=5, slices=4, seed=seed)
+        except ns["Hazard"]:
+            caught += 1
+    assert caught > 0
