@@ -158,12 +158,13 @@ Splits decode_splits(const State& s) {
     const rma_config& c = s.cfg;
     int want_r = s.ring_splits_override, want_b = s.bank_splits_override;
     if (want_r <= 0 || want_b <= 0) {
-        // one CTA per SM at a time: about four waves of CTAs, without cutting rows so
-        // thin that the per-split merge dominates (at most 8 + 8 splits, 128 rows each
-        // for the pages' ring and bank)
+        // One CTA per SM at a time.  From 16 (sequence, group) units up, about half a wave of CTAs:
+        // the tensor-core kernel streams a split fast enough that fewer, longer splits (less merging)
+        // win; a batch of 1 or 2 is latency bound and takes the most splits (8 + 8, 128 rows each
+        // for the pages' ring and bank).
         const long units = (long)c.batch * c.n_groups;
-        const long target = (long)s.sm_count * 4;
-        long per_unit = (target + units - 1) / units;
+        const long target = (long)s.sm_count / 2;
+        long per_unit = units <= 8 ? 16 : (target + units - 1) / units;
         if (per_unit < 2) per_unit = 2;
         if (per_unit > 16) per_unit = 16;
         want_r = (int)(per_unit / 2);
