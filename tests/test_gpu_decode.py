@@ -59,8 +59,9 @@ def test_tiny_decode_config_full_parity():
     print(f"tiny decode: worst output error {worst:.3e}")
 
 
-# None is the default shape for this batch; (5, 5), (2, 3), (1, 2) and (8, 8) are the defaults the
-# split heuristic picks at other batch sizes (ragged batch 32 / 64 / 128 sweeps, batch 1)
+# None is the default shape for this batch; (1, 1), (2, 3) and (8, 8) are the defaults the split
+# heuristic picks at other batch sizes (16 and up, 8, and 1 or 2); (5, 5) and (1, 2) were earlier
+# defaults and stay as extra shapes
 @pytest.mark.parametrize("splits", [None, (1, 1), (3, 5), (16, 16), (32, 32), (1, 63), (5, 5), (2, 3), (1, 2), (8, 8)])
 def test_ragged_fills_every_split_shape(splits):
     """Partial windows, empty and partial banks, pending about to fill; quantised scores force ties."""
