@@ -71,8 +71,9 @@ extern "C" {
  * [0, bank_slots], pend_fill not in [0, pend_slots]), e.g. a corrupted restore:
  * it clamped them for its own indexing and went on. */
 #define RMA_STATUS_BAD_COUNTERS              8u
-/* A kernel gave up waiting on one of its own pipeline barriers (a bounded
- * wait of about two seconds ran out) and abandoned its tile; its outputs are
+/* A kernel gave up waiting on one of its own pipeline barriers, or a prefill
+ * commit CTA on the attention launch's rows of its group (a bounded wait of
+ * about two seconds ran out), and abandoned its work; its outputs are
  * not valid, and the state of the groups it served (slots, counters,
  * tickets) may be inconsistent: restore the state buffer from a copy or lay
  * it out afresh with rma_state_alloc before the next call on it.  Indicates
