@@ -14,8 +14,9 @@
 //
 // 1. prefill_attn_kernel, persistent: clusters of 2 CTAs, one CTA per SM, as
 //    few as keep the most items per cluster at its minimum (the SMs left over
-//    run the commit of finished groups), each looping over work items.  An item is one (sequence, group,
-//    pair of tiles, phase): a tile is 32 tokens x the group's 4 query heads =
+//    run the commit of finished groups), each looping over work items.  An
+//    item is one (sequence, group, pair of tiles, phase): a tile is 32 tokens
+//    x the group's 4 query heads =
 //    128 query rows, the two tiles of a pair are the two CTAs of a tcgen05
 //    cta_group::2 MMA pair (M = 256; both read exactly the same keys, so each
 //    CTA loads only half of every 64-key K/V chunk), and the phase is the local
@@ -51,8 +52,8 @@
 //    first launch), wait until every item of their group has stored its rows
 //    (each softmax warp counts its rows of an item in the high half of the
 //    group's ticket word once its TMA stores have completed; items run in
-//    group-major order, so
-//    most groups are done well before the last), then combine out = local +
+//    group-major order, so most groups are done well before the last), then
+//    combine out = local +
 //    gate * anchor in FP32, rounded once to BF16, and write the block's K/V into
 //    the ring (every read of the group's ring is done); one CTA runs the forced
 //    admit's competition (scores only, no wait) and leaves the list of admitted
@@ -112,7 +113,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct Tmaps {
     CUtensorMap k, v, ring_k, ring_v, bank_k, bank_v;   // K maps: 32-row boxes; V maps: 64-row boxes
-    CUtensorMap ws;   // FP32 [phase][b][t][head][256], boxes of 32 dims x 4 heads x 32 tokens
+    CUtensorMap ws;   // FP32 [phase][b][t][head][256], boxes of 32 dims x 4 heads x 8 tokens (one warp's rows)
 };
 
 enum Bar {
@@ -1003,7 +1004,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d1, uint64_t d2, uint64
 }
 
 // The FP32 workspace [phase 2][b B][t n][head HQ][256] for TMA stores: boxes of 32 dims x 4 heads
-// x 32 tokens, 128-byte swizzle (the rows' 16-byte pieces permuted by row within 8-row groups).
+// x 8 tokens (one softmax warp's 32 rows), 128-byte swizzle (the rows' 16-byte pieces permuted by
+// row within 8-row groups).
 bool make_ws_map(CUtensorMap* m, void* ws, int HQ, int n, int B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
